@@ -1,0 +1,317 @@
+"""Pins for the fp64 oracle, each against something other than the oracle itself.
+
+* brute force with numpy/scipy library routines on tiny inputs,
+* closed forms (equal keys, zero queries, a planted dominant logit, causal row 0),
+* the two-chunk parity harness of "DeDLOC Guide", Step 4 (merge of two
+  chunks' (O, LSE) equals dense attention over their union),
+* ring == dense for many P and both chunk orders,
+* merge order independence and the empty-partial (-inf) rule,
+* gradients: central finite differences, torch fp64 autograd, and the
+  identities sum_j dK_j = 0 and sum_j dV_j = sum_i dO_i,
+* hand-derived rank-major maps and ring schedules from tests/golden/.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+from scipy.special import logsumexp
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _np_attention(q, k, v, causal, scale):
+    """Textbook dense attention with numpy/scipy (independent of the oracle)."""
+    B, H, S, D = q.shape
+    Hkv, Sk = k.shape[1], k.shape[2]
+    G = H // Hkv
+    o = np.zeros((B, H, S, D))
+    lse = np.zeros((B, H, S))
+    for b in range(B):
+        for h in range(H):
+            s = scale * q[b, h] @ k[b, h // G].T
+            if causal:
+                mask = np.arange(Sk)[None, :] > np.arange(S)[:, None]
+                s = np.where(mask, -np.inf, s)
+            lse[b, h] = logsumexp(s, axis=-1)
+            w = np.exp(s - lse[b, h][:, None])
+            o[b, h] = w @ v[b, h // G]
+    return o, lse
+
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("H,Hkv", [(1, 1), (4, 2), (4, 1), (3, 3)])
+@pytest.mark.parametrize("S,D", [(1, 1), (5, 3), (16, 8), (9, 4)])
+def test_forward_matches_numpy_bruteforce(causal, H, Hkv, S, D):
+    seed = hash((causal, H, Hkv, S, D)) % 2**31
+    q, k, v = _rand((2, H, S, D), seed), _rand((2, Hkv, S, D), seed + 1), _rand((2, Hkv, S, D), seed + 2)
+    scale = 1 / math.sqrt(D)
+    o, lse = oracle.attn_fwd(q, k, v, causal, scale)
+    o_ref, lse_ref = _np_attention(q, k, v, causal, scale)
+    np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=1e-13)
+
+
+def test_forward_row_subset_and_scale_argument():
+    q, k, v = _rand((1, 2, 12, 4), 1), _rand((1, 2, 12, 4), 2), _rand((1, 2, 12, 4), 3)
+    rows = np.array([0, 5, 11])
+    o_all, lse_all = oracle.attn_fwd(q, k, v, True, 0.3)
+    o, lse = oracle.attn_fwd(q, k, v, True, 0.3, rows=rows)
+    np.testing.assert_array_equal(o, o_all[:, :, rows])
+    np.testing.assert_array_equal(lse, lse_all[:, :, rows])
+    o_ref, lse_ref = _np_attention(q, k, v, True, 0.3)
+    np.testing.assert_allclose(lse_all, lse_ref, atol=1e-13, rtol=0)
+
+
+def test_closed_form_equal_keys():
+    # all keys equal: every visible score is s = scale <q_i, k>, so attention is
+    # the mean of the visible values and LSE = s + ln |V(i)|.
+    S, D = 10, 4
+    q = _rand((1, 1, S, D), 5)
+    kvec = _rand((D,), 6)
+    k = np.broadcast_to(kvec, (1, 1, S, D)).copy()
+    v = _rand((1, 1, S, D), 7)
+    scale = 0.7
+    for causal in (False, True):
+        o, lse = oracle.attn_fwd(q, k, v, causal, scale)
+        for i in range(S):
+            n = i + 1 if causal else S
+            s = scale * q[0, 0, i] @ kvec
+            np.testing.assert_allclose(o[0, 0, i], v[0, 0, :n].mean(axis=0), atol=1e-14)
+            assert abs(lse[0, 0, i] - (s + math.log(n))) < 1e-13
+
+
+def test_closed_form_zero_queries_and_causal_row0():
+    S, D = 8, 3
+    q = np.zeros((1, 1, S, D))
+    k, v = _rand((1, 1, S, D), 8), _rand((1, 1, S, D), 9)
+    o, lse = oracle.attn_fwd(q, k, v, False, 1.0)
+    np.testing.assert_allclose(o[0, 0], np.broadcast_to(v[0, 0].mean(0), (S, D)), atol=1e-14)
+    np.testing.assert_allclose(lse[0, 0], math.log(S), atol=1e-14)
+    # causal row 0 sees only key 0: O_0 = v_0, LSE_0 = s_00
+    q = _rand((1, 1, S, D), 10)
+    o, lse = oracle.attn_fwd(q, k, v, True, 0.5)
+    np.testing.assert_allclose(o[0, 0, 0], v[0, 0, 0], atol=1e-15)
+    assert abs(lse[0, 0, 0] - 0.5 * q[0, 0, 0] @ k[0, 0, 0]) < 1e-14
+
+
+def test_closed_form_dominant_logit():
+    # one key aligned with the query at a huge logit: softmax is one-hot.
+    S, D = 6, 4
+    q = np.zeros((1, 1, S, D)); q[0, 0, :, 0] = 1.0
+    k = np.zeros((1, 1, S, D)); k[0, 0, 3, 0] = 1000.0
+    v = _rand((1, 1, S, D), 11)
+    o, lse = oracle.attn_fwd(q, k, v, False, 1.0)
+    np.testing.assert_allclose(o[0, 0], np.broadcast_to(v[0, 0, 3], (S, D)), atol=1e-14)
+    np.testing.assert_allclose(lse[0, 0], 1000.0, atol=1e-12)
+
+
+def test_two_chunk_merge_harness():
+    # "DeDLOC Guide", Step 4: attention over KV chunk 0 and chunk 1 separately,
+    # merged, equals dense attention over both (B=1, H=8, 64 queries, 64+64 keys,
+    # D=64, fp32 there with max-abs < 1e-5; fp64 here).
+    B, H, S, D = 1, 8, 64, 64
+    q = _rand((B, H, S, D), 12)
+    k0, v0 = _rand((B, H, S, D), 13), _rand((B, H, S, D), 14)
+    k1, v1 = _rand((B, H, S, D), 15), _rand((B, H, S, D), 16)
+    scale = 1 / math.sqrt(D)
+    o0, l0 = oracle.attn_fwd(q, k0, v0, False, scale)
+    o1, l1 = oracle.attn_fwd(q, k1, v1, False, scale)
+    om, lm = oracle.lse_merge(o0.reshape(-1, D), l0.reshape(-1), o1.reshape(-1, D), l1.reshape(-1))
+    kf, vf = np.concatenate([k0, k1], axis=2), np.concatenate([v0, v1], axis=2)
+    o_ref, lse_ref = _np_attention(q, kf, vf, False, scale)
+    assert np.abs(om.reshape(o_ref.shape) - o_ref).max() < 1e-12
+    assert np.abs(lm.reshape(lse_ref.shape) - lse_ref).max() < 1e-12
+    # and the oracle's own dense path over the concatenation agrees too
+    od, ld = oracle.attn_fwd(q, kf, vf, False, scale)
+    assert np.abs(od - o_ref).max() < 1e-13
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("order", [oracle.CONTIGUOUS, oracle.ZIGZAG])
+@pytest.mark.parametrize("P", [1, 2, 3, 4, 8])
+def test_ring_equals_dense(causal, order, P):
+    S = 48 if P == 3 else 32
+    H, Hkv, D = 4, 2, 8
+    q, k, v = _rand((1, H, S, D), 17 + P), _rand((1, Hkv, S, D), 18), _rand((1, Hkv, S, D), 19)
+    o_d, l_d = oracle.attn_fwd(q, k, v, causal)
+    o_r, l_r = oracle.ring_fwd(q, k, v, causal, P, order)
+    assert np.abs(o_r - o_d).max() < 1e-12
+    assert np.abs(l_r - l_d).max() < 1e-12
+
+
+def test_ring_zigzag_equals_contiguous_after_unpermute():
+    # The orders only move tokens between ranks; in natural order the results agree.
+    S, D, P = 64, 4, 4
+    q, k, v = _rand((1, 2, S, D), 20), _rand((1, 2, S, D), 21), _rand((1, 2, S, D), 22)
+    oz, lz = oracle.ring_fwd(q, k, v, True, P, oracle.ZIGZAG)
+    oc, lc = oracle.ring_fwd(q, k, v, True, P, oracle.CONTIGUOUS)
+    assert np.abs(oz - oc).max() < 1e-12 and np.abs(lz - lc).max() < 1e-12
+
+
+def test_merge_order_independence_and_empty_partials():
+    rng = np.random.default_rng(23)
+    n, rows, D = 6, 5, 7
+    parts = [(rng.standard_normal((rows, D)), rng.standard_normal(rows) * 3) for _ in range(n)]
+    # one partial is empty on some rows: (0, -inf) is the identity
+    parts[2][1][1] = -np.inf
+    parts[2][0][1] = 0.0
+
+    def fold(order):
+        o, l = parts[order[0]][0].copy(), parts[order[0]][1].copy()
+        for idx in order[1:]:
+            o, l = oracle.lse_merge(o, l, parts[idx][0], parts[idx][1])
+        return o, l
+
+    ref_o, ref_l = fold(list(range(n)))
+    for perm in list(itertools.permutations(range(n)))[::37]:
+        o, l = fold(list(perm))
+        assert np.abs(o - ref_o).max() < 1e-12 and np.abs(l - ref_l).max() < 1e-12
+    # tree-shaped merge
+    a = oracle.lse_merge(*fold([0, 1]), *fold([2, 3]))
+    t = oracle.lse_merge(*a, *fold([4, 5]))
+    assert np.abs(t[0] - ref_o).max() < 1e-12 and np.abs(t[1] - ref_l).max() < 1e-12
+    # closed form of the merge: partials over disjoint sets merge to softmax over the union
+    w = np.exp(np.stack([p[1] for p in parts]))           # per-partial normaliser
+    o_cf = sum(wi[:, None] * p[0] for wi, p in zip(w, parts)) / w.sum(0)[:, None]
+    assert np.abs(ref_o - o_cf).max() < 1e-12
+    assert np.abs(ref_l - np.log(w.sum(0))).max() < 1e-12
+    # both empty -> (0, -inf), never NaN
+    o, l = oracle.lse_merge(np.ones((1, D)), np.array([-np.inf]), np.ones((1, D)), np.array([-np.inf]))
+    assert np.all(o == 0) and l[0] == -np.inf
+
+
+def _loss(q, k, v, dout, causal, scale):
+    o, _ = oracle.attn_fwd(q, k, v, causal, scale)
+    return float((o * dout).sum())
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_finite_differences(causal):
+    B, H, Hkv, S, D = 1, 4, 2, 12, 4
+    q, k, v = _rand((B, H, S, D), 24), _rand((B, Hkv, S, D), 25), _rand((B, Hkv, S, D), 26)
+    dout = _rand((B, H, S, D), 27)
+    scale = 1 / math.sqrt(D)
+    dq, dkv = oracle.attn_bwd(q, k, v, dout, causal, scale)
+    h = 1e-6
+    rng = np.random.default_rng(28)
+    for name, x in (("q", q), ("k", k), ("v", v)):
+        for _ in range(12):
+            idx = tuple(rng.integers(0, n) for n in x.shape)
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args = {"q": q, "k": k, "v": v}
+            args[name] = xp
+            lp = _loss(args["q"], args["k"], args["v"], dout, causal, scale)
+            args[name] = xm
+            lm = _loss(args["q"], args["k"], args["v"], dout, causal, scale)
+            fd = (lp - lm) / (2 * h)
+            b, hh, s, d = idx
+            if name == "q":
+                an = dq[(b, hh)][s, d]
+            elif name == "k":
+                an = dkv[(b, hh)][0][s, d]
+            else:
+                an = dkv[(b, hh)][1][s, d]
+            assert abs(fd - an) <= 1e-7 * max(1.0, abs(an)), (name, idx, fd, an)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_matches_torch_autograd(causal):
+    B, H, Hkv, S, D = 2, 4, 1, 10, 6
+    q, k, v = _rand((B, H, S, D), 29), _rand((B, Hkv, S, D), 30), _rand((B, Hkv, S, D), 31)
+    dout = _rand((B, H, S, D), 32)
+    scale = 0.37
+    tq, tk, tv = (torch.tensor(a, requires_grad=True) for a in (q, k, v))
+    G = H // Hkv
+    kk = tk.repeat_interleave(G, dim=1)
+    vv = tv.repeat_interleave(G, dim=1)
+    s = torch.matmul(tq, kk.transpose(-1, -2)) * scale
+    if causal:
+        s = s.masked_fill(torch.triu(torch.ones(S, S, dtype=torch.bool), 1), float("-inf"))
+    o = torch.matmul(torch.softmax(s, -1), vv)
+    (o * torch.tensor(dout)).sum().backward()
+    dq, dkv = oracle.attn_bwd(q, k, v, dout, causal, scale)
+    for b in range(B):
+        for h in range(H):
+            np.testing.assert_allclose(dq[(b, h)], tq.grad[b, h].numpy(), atol=1e-12, rtol=0)
+        for g in range(Hkv):
+            np.testing.assert_allclose(dkv[(b, g)][0], tk.grad[b, g].numpy(), atol=1e-12, rtol=0)
+            np.testing.assert_allclose(dkv[(b, g)][1], tv.grad[b, g].numpy(), atol=1e-12, rtol=0)
+
+
+def test_backward_identities_and_row_subsets():
+    # sum_j dS_ij = 0 per query row, hence sum_j dK_j = 0; softmax rows sum to
+    # one, hence sum_j dV_j = sum_i dO_i (per KV head, summed over its group).
+    B, H, Hkv, S, D = 1, 2, 1, 20, 5
+    q, k, v = _rand((B, H, S, D), 33), _rand((B, Hkv, S, D), 34), _rand((B, Hkv, S, D), 35)
+    dout = _rand((B, H, S, D), 36)
+    for causal in (False, True):
+        dq, dkv = oracle.attn_bwd(q, k, v, dout, causal)
+        dk, dv = dkv[(0, 0)]
+        assert np.abs(dk.sum(0)).max() < 1e-12
+        np.testing.assert_allclose(dv.sum(0), dout[0].sum(axis=(0, 1)), atol=1e-12)
+        rows = np.array([3, 7, 19])
+        dq_s, dkv_s = oracle.attn_bwd(q, k, v, dout, causal, qrows=rows, krows=rows,
+                                      heads=([(0, 1)], [(0, 0)]))
+        np.testing.assert_allclose(dq_s[(0, 1)], dq[(0, 1)][rows], atol=1e-13)
+        np.testing.assert_allclose(dkv_s[(0, 0)][0], dk[rows], atol=1e-13)
+        np.testing.assert_allclose(dkv_s[(0, 0)][1], dv[rows], atol=1e-13)
+
+
+def _golden_lines(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                lhs, rhs = line.split(":")
+                yield lhs.split(), [int(x) for x in rhs.split()]
+
+
+def test_rank_major_positions_golden():
+    n = 0
+    for (order, S, P), expect in _golden_lines("rank_major_positions.txt"):
+        o = oracle.ZIGZAG if order == "zigzag" else oracle.CONTIGUOUS
+        assert list(oracle.rank_major_positions(int(S), int(P), o)) == expect
+        n += 1
+    assert n >= 6
+
+
+def test_ring_schedule_golden():
+    n = 0
+    for (P, i), expect in _golden_lines("ring_schedule.txt"):
+        assert [oracle.ring_owner(int(P), int(i), t) for t in range(int(P))] == expect
+        n += 1
+    assert n >= 5
+
+
+@pytest.mark.parametrize("S,P", [(64, 4), (96, 3), (1024, 8), (32, 16)])
+def test_rank_major_positions_bijection_and_roundtrip(S, P):
+    for order in (oracle.CONTIGUOUS, oracle.ZIGZAG):
+        pos = oracle.rank_major_positions(S, P, order)
+        assert sorted(pos.tolist()) == list(range(S))
+        x = np.arange(S * 3).reshape(1, S, 3)
+        assert np.array_equal(oracle.to_natural(oracle.to_rank_major(x, P, order, 1), P, order, 1), x)
+    with pytest.raises(ValueError):
+        oracle.rank_major_positions(S + 1, P, oracle.ZIGZAG)
+
+
+def test_ulysses_layout_is_a_bijection():
+    B, S, H, D = 2, 12, 4, 3
+    src = np.arange(B * S * H * D).reshape(B, S, H, D)
+    dst = oracle.ulysses_seq_to_head(src)
+    assert dst.shape == (B, H, S, D)
+    # every element lands exactly once, at [b, h, s, d] <- [b, s, h, d]
+    assert sorted(dst.ravel().tolist()) == list(range(src.size))
+    for b, s, h, d in [(0, 0, 0, 0), (1, 11, 3, 2), (0, 5, 2, 1)]:
+        assert dst[b, h, s, d] == src[b, s, h, d]
+    assert np.array_equal(oracle.ulysses_head_to_seq(dst), src)
