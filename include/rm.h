@@ -1,0 +1,200 @@
+/*
+ * rm.h — C ABI of the B200 (sm_100a) blockwise ring attention library.
+ *
+ * What it computes. P virtual sequence-parallel ranks are simulated on one GPU.
+ * Each rank keeps its query block fixed while the key/value blocks travel
+ * around the ring ("Sequence Parallelism III: Ring Attention for Context That
+ * Does Not Fit", duoan.github.io LLM tag index). Every step runs a flash-style
+ * tile pass (QK^T, causal mask, online softmax, PV). Its partial output and
+ * log-sum-exp fold into a running (O, LSE) pair by max-shifted exponential
+ * weights ("DeDLOC Guide: Decentralized Long-Context Attention", section 3,
+ * Online Softmax Rescaling Across Decentralized Ranks; Step 3, the local step
+ * and the merge). The ring's block rotation is HBM block indexing: at step t
+ * rank i reads the key/value block of owner (i - t) mod P.
+ *
+ * Conventions for every entry point:
+ *   - All tensor arguments are DEVICE pointers owned by the caller; the library
+ *     never allocates device memory and keeps no pointer after it returns.
+ *   - Calls are asynchronous on `stream` (0 = legacy default stream). Inputs
+ *     must stay valid, and outputs untouched, until the stream reaches the work.
+ *   - Tensors are dense row-major. Attention tensors are [B, heads, S, D] with
+ *     the S axis RANK-MAJOR: rank 0's L = S/P tokens, then rank 1's, and so
+ *     on, each rank's tokens in its local chunk order (see rm_order).
+ *   - Host-side validation runs before any launch; on RM_ERR_INVALID_ARG or
+ *     RM_ERR_UNSUPPORTED nothing is launched and nothing is written.
+ *   - Empty problems (B == 0 or S == 0, rows == 0) are valid and do nothing.
+ *   - Pointers must be 16-byte aligned (TMA and vector access).
+ *   - A launch failure returns RM_ERR_CUDA; rm_last_cuda_error() then gives the
+ *     cudaError_t of the calling thread's last failure.
+ *   - Every wait inside a kernel is bounded (see rm_set_watchdog_ns). A wait that
+ *     runs out makes the kernel stop early, write nothing further and set a
+ *     device status word that rm_check_device_status() reports as
+ *     RM_ERR_TIMEOUT. Outputs of such a call are undefined.
+ */
+#ifndef RM_H
+#define RM_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define RM_API __attribute__((visibility("default")))
+#else
+#define RM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum rm_status {
+    RM_OK = 0,
+    RM_ERR_INVALID_ARG = 1,  /* null pointer, bad size, bad enum, misalignment */
+    RM_ERR_UNSUPPORTED = 2,  /* valid request outside the shapes/dtypes built */
+    RM_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+    RM_ERR_TIMEOUT = 4       /* a bounded in-kernel wait ran out */
+} rm_status;
+
+/* Token order of the ring ("context parallelism", Last Dictionary: causal
+ * imbalance is handled by reordering chunks; axolotl-ringmaster README,
+ * Layout: balancers.py head_tail/contiguous index generation).
+ *   CONTIGUOUS: rank i holds natural tokens [i*L, (i+1)*L), L = S/P.
+ *   ZIGZAG:     the sequence is cut into 2P chunks of c = S/(2P); rank i holds
+ *               chunk i followed by chunk 2P-1-i (balances causal work). */
+typedef enum rm_order { RM_ORDER_CONTIGUOUS = 0, RM_ORDER_ZIGZAG = 1 } rm_order;
+
+typedef enum rm_dtype { RM_DTYPE_BF16 = 0, RM_DTYPE_FP32 = 1 } rm_dtype;
+
+typedef enum rm_permute_dir { RM_SEQ_TO_HEAD = 0, RM_HEAD_TO_SEQ = 1 } rm_permute_dir;
+
+typedef enum rm_reorder_dir {
+    RM_NATURAL_TO_RANK_MAJOR = 0,
+    RM_RANK_MAJOR_TO_NATURAL = 1
+} rm_reorder_dir;
+
+/*
+ * rm_ring_attn_fwd — ring attention forward over P virtual ranks.
+ *
+ * Follows "DeDLOC Guide", Step 3 (scores = scale * Q K^T, LSE = logsumexp over
+ * keys, O = softmax * V) run blockwise with the online-softmax merge of
+ * section 3, and the Best Practices table's "Causal Mask Handling" (whole
+ * masked blocks are skipped). Causal visibility uses GLOBAL token positions:
+ * key j is visible to query i iff pos(j) <= pos(i) (diagonal included).
+ *
+ *   q    [B, H,   S, D]  dtype            (rank-major S)
+ *   k, v [B, Hkv, S, D]  dtype; query head h reads KV head h / (H/Hkv)
+ *   o    [B, H,   S, D]  dtype, written
+ *   lse  [B, H,   S]     float32, written: natural log of sum_j exp(scale*q.k_j)
+ *   scale > 0 (usually 1/sqrt(D)).
+ *
+ * Supported: dtype BF16 (tensor cores, fp32 accumulation) or FP32 (exact fp32
+ * FMA path); D in {64, 128}; H % Hkv == 0; P >= 1; ZIGZAG needs S % (2P*128)
+ * == 0, CONTIGUOUS needs S % (P*256) == 0 (for FP32: S % (2P*64) == 0 and
+ * S % (P*64) == 0 respectively). Other shapes return RM_ERR_UNSUPPORTED.
+ */
+RM_API rm_status rm_ring_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                           int B, int H, int Hkv, int S, int D, int P, int causal,
+                           rm_order order, rm_dtype dtype, float scale, cudaStream_t stream);
+
+/*
+ * rm_ring_attn_bwd — gradients of L = sum(dO * O) through the ring forward
+ * (axolotl-ringmaster README: flash-style reverse-ring backward; gradients
+ * accumulate in fp32 across ring steps).
+ *
+ * With P_ij = exp(scale*q_i.k_j - LSE_i) over visible keys and
+ * Delta_i = <dO_i, O_i>: dV_j = sum_i P_ij dO_i, dS_ij = P_ij (<dO_i, v_j> -
+ * Delta_i), dQ_i = scale sum_j dS_ij k_j, dK_j = scale sum_i dS_ij q_i; a KV
+ * head's dK/dV sum over the query heads that share it.
+ *
+ *   q, k, v, o, dout : as in the forward (dtype; o is the forward's output)
+ *   lse              : [B, H, S] float32 from the forward
+ *   dq [B,H,S,D], dk, dv [B,Hkv,S,D] : float32, overwritten (zeroed first by
+ *                      the library)
+ *   workspace        : device scratch of at least
+ *                      rm_ring_attn_bwd_workspace_size(B, H, S) bytes, 256-byte
+ *                      aligned, owned by the caller, contents need not be set.
+ * Supported: dtype BF16, D in {64, 128}, same shape rules as the forward.
+ */
+RM_API size_t rm_ring_attn_bwd_workspace_size(int B, int H, int S);
+
+RM_API rm_status rm_ring_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                           const float* lse, const void* dout, float* dq, float* dk,
+                           float* dv, void* workspace, size_t workspace_bytes, int B, int H,
+                           int Hkv, int S, int D, int P, int causal, rm_order order,
+                           rm_dtype dtype, float scale, cudaStream_t stream);
+
+/*
+ * rm_lse_merge — fold one partial (O, LSE) into a running pair, row by row,
+ * in place ("DeDLOC Guide", section 3 alpha/beta rescaling, in the
+ * normalised-output form of Step 3's merge):
+ *   M = max(a, b); if M = -inf: O = 0, LSE = -inf (empty + empty);
+ *   else wa = exp(a - M), wb = exp(b - M),
+ *        O = (wa O_acc + wb O_part) / (wa + wb), LSE = M + ln(wa + wb).
+ *   o_acc [rows, D] f32 (in/out), lse_acc [rows] f32 (in/out),
+ *   o_part [rows, D] f32, lse_part [rows] f32. D >= 1, rows >= 0.
+ */
+RM_API rm_status rm_lse_merge(float* o_acc, float* lse_acc, const float* o_part, const float* lse_part,
+                       int64_t rows, int D, cudaStream_t stream);
+
+/*
+ * rm_ulysses_permute — the DeepSpeed-Ulysses all-to-all as a layout transform
+ * on one device ("Sequence Parallelism II: DeepSpeed Ulysses and All-to-All
+ * Attention", duoan.github.io LLM tag index: before the exchange every rank
+ * has all heads for a subset of tokens, after it all tokens for a subset of
+ * heads; axolotl-ringmaster README: Ulysses is capped by the KV-head count).
+ *
+ * Mesh: U Ulysses ranks x R ring ranks; shard n = r*U + u holds tokens
+ * [n*S/(U R), (n+1)*S/(U R)) of the rank-major sequence.
+ *   SEQ_TO_HEAD: src [B, S, Hx, D] (= [B, U*R shards, S/(U R), Hx, D]) ->
+ *                dst [B, Hx, S, D]; device (r, u)'s share afterwards is heads
+ *                [u*Hx/U, (u+1)*Hx/U) x tokens [r*S/R, (r+1)*S/R).
+ *   HEAD_TO_SEQ: the exact inverse.
+ * Requires Hx % U == 0, S % (U*R) == 0, elem_bytes in {1, 2, 4, 8}.
+ * Bit-exact data movement.
+ */
+RM_API rm_status rm_ulysses_permute(const void* src, void* dst, int B, int S, int Hx, int D, int U,
+                             int R, int elem_bytes, rm_permute_dir dir, cudaStream_t stream);
+
+/* As rm_ulysses_permute for Q (H heads) and K, V (Hkv heads) in ONE launch
+ * (axolotl-ringmaster README: the Ulysses leg fuses K/V into one exchange).
+ * Requires H % U == 0, Hkv % U == 0 (so U <= Hkv). */
+RM_API rm_status rm_ulysses_permute_qkv(const void* q_src, const void* k_src, const void* v_src,
+                                 void* q_dst, void* k_dst, void* v_dst, int B, int S, int H,
+                                 int Hkv, int D, int U, int R, int elem_bytes,
+                                 rm_permute_dir dir, cudaStream_t stream);
+
+/*
+ * rm_seq_reorder — natural token order <-> rank-major ring order along S.
+ *   src, dst [B, H, S, D] elements of elem_bytes each (D = 1 for LSE).
+ *   NATURAL_TO_RANK_MAJOR: dst[.., s, :] = src[.., pos(s), :]
+ *   RANK_MAJOR_TO_NATURAL: dst[.., pos(s), :] = src[.., s, :]
+ * pos(s) as in rm_order. Requires S % P == 0 (contiguous) or S % (2P) == 0
+ * (zigzag). src and dst must not overlap. Bit-exact.
+ */
+RM_API rm_status rm_seq_reorder(const void* src, void* dst, int B, int H, int S, int D, int P,
+                         rm_order order, rm_reorder_dir dir, int elem_bytes,
+                         cudaStream_t stream);
+
+/* Synchronises `stream`, then reads and clears the device status word of the
+ * current device. Returns RM_ERR_TIMEOUT if a bounded wait ran out since the
+ * last check, RM_ERR_CUDA if the synchronisation failed, else RM_OK. */
+RM_API rm_status rm_check_device_status(cudaStream_t stream);
+
+/* Limit for every in-kernel wait, in nanoseconds (default 2e9). Applies to
+ * launches made after the call; values below 1000 are raised to 1000. */
+RM_API void rm_set_watchdog_ns(uint64_t ns);
+
+/* Launches one kernel that waits on a barrier nothing will complete, bounded
+ * by timeout_ns, so that callers can see the watchdog path end in
+ * RM_ERR_TIMEOUT (reported by rm_check_device_status) without a hang. */
+RM_API rm_status rm_watchdog_selftest(uint64_t timeout_ns, cudaStream_t stream);
+
+RM_API const char* rm_status_string(rm_status status);
+RM_API int rm_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RM_H */

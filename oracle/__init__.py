@@ -64,6 +64,10 @@ def _L():
 
 
 def _f64(a):
+    """Exact widening to contiguous float64 (numpy or torch input)."""
+    if hasattr(a, "detach"):  # torch tensor: bf16/fp32 -> fp64 exactly
+        import torch
+        a = a.detach().to("cpu", torch.float64).numpy()
     return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
 
 
@@ -73,6 +77,18 @@ def _i64(a):
 
 def _p(a, t=ctypes.c_double):
     return a.ctypes.data_as(ctypes.POINTER(t))
+
+
+def _shape(a):
+    return tuple(a.shape)
+
+
+def _rows_of(x, r):
+    """Rows r (int64 numpy) of a 2-D numpy array or torch tensor."""
+    if hasattr(x, "index_select"):
+        import torch
+        return x.index_select(0, torch.from_numpy(r))
+    return x[r]
 
 
 def num_threads() -> int:
@@ -150,14 +166,14 @@ def _rows_arg(rows, S):
 def attn_fwd(q, k, v, causal: bool, scale: float = None, rows=None):
     """Dense softmax attention in natural order.
 
-    q [B,H,S,D], k/v [B,Hkv,Sk,D]; query head h reads KV head h // (H/Hkv).
+    q [B,H,S,D], k/v [B,Hkv,Sk,D] (numpy or torch, any float dtype; widened to
+    fp64 one head at a time); query head h reads KV head h // (H/Hkv).
     rows: natural query positions to evaluate (same for every head), or None
     for all. Returns O [B,H,n,D] and LSE [B,H,n] (natural log of the scaled
     scores), float64.
     """
-    q, k, v = _f64(q), _f64(k), _f64(v)
-    B, H, S, D = q.shape
-    Hkv, Sk = k.shape[1], k.shape[2]
+    B, H, S, D = _shape(q)
+    Hkv, Sk = _shape(k)[1], _shape(k)[2]
     G = H // Hkv
     scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
     r = _rows_arg(rows, S)
@@ -165,15 +181,15 @@ def attn_fwd(q, k, v, causal: bool, scale: float = None, rows=None):
     lse = np.zeros((B, H, len(r)))
     lib = _L()
     for b in range(B):
-        for h in range(H):
-            qh = np.ascontiguousarray(q[b, h])
-            kh = np.ascontiguousarray(k[b, h // G])
-            vh = np.ascontiguousarray(v[b, h // G])
-            ob = np.zeros((len(r), D))
-            lb = np.zeros(len(r))
-            lib.orc_attn_fwd_head(_p(qh), _p(kh), _p(vh), Sk, D, int(causal), scale,
-                                  _p(r, ctypes.c_int64), len(r), _p(ob), _p(lb))
-            o[b, h], lse[b, h] = ob, lb
+        for g in range(Hkv):
+            kh, vh = _f64(k[b, g]), _f64(v[b, g])
+            for h in range(g * G, (g + 1) * G):
+                qh = _f64(_rows_of(q[b, h], r) if rows is not None else q[b, h])
+                ob = np.zeros((len(r), D))
+                lb = np.zeros(len(r))
+                lib.orc_attn_fwd_head(_p(qh), _p(kh), _p(vh), Sk, D, int(causal), scale,
+                                      _p(r, ctypes.c_int64), len(r), _p(ob), _p(lb))
+                o[b, h], lse[b, h] = ob, lb
     return o, lse
 
 
@@ -183,9 +199,8 @@ def ring_fwd(q, k, v, causal: bool, P: int, order: int, scale: float = None, row
     Same arguments and results as attn_fwd (natural order in and out); the
     ring layout only decides which keys each step's partial covers.
     """
-    q, k, v = _f64(q), _f64(k), _f64(v)
-    B, H, S, D = q.shape
-    Hkv = k.shape[1]
+    B, H, S, D = _shape(q)
+    Hkv = _shape(k)[1]
     G = H // Hkv
     scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
     r = _rows_arg(rows, S)
@@ -193,15 +208,15 @@ def ring_fwd(q, k, v, causal: bool, P: int, order: int, scale: float = None, row
     lse = np.zeros((B, H, len(r)))
     lib = _L()
     for b in range(B):
-        for h in range(H):
-            qh = np.ascontiguousarray(q[b, h])
-            kh = np.ascontiguousarray(k[b, h // G])
-            vh = np.ascontiguousarray(v[b, h // G])
-            ob = np.zeros((len(r), D))
-            lb = np.zeros(len(r))
-            lib.orc_ring_fwd_head(_p(qh), _p(kh), _p(vh), S, D, int(causal), scale, P,
-                                  order, _p(r, ctypes.c_int64), len(r), _p(ob), _p(lb))
-            o[b, h], lse[b, h] = ob, lb
+        for g in range(Hkv):
+            kh, vh = _f64(k[b, g]), _f64(v[b, g])
+            for h in range(g * G, (g + 1) * G):
+                qh = _f64(_rows_of(q[b, h], r) if rows is not None else q[b, h])
+                ob = np.zeros((len(r), D))
+                lb = np.zeros(len(r))
+                lib.orc_ring_fwd_head(_p(qh), _p(kh), _p(vh), S, D, int(causal), scale, P,
+                                      order, _p(r, ctypes.c_int64), len(r), _p(ob), _p(lb))
+                o[b, h], lse[b, h] = ob, lb
     return o, lse
 
 
@@ -227,9 +242,8 @@ def attn_bwd(q, k, v, dout, causal: bool, scale: float = None, qrows=None,
     (b, h) -> dQ [nq, D] and (b, g) -> (dK [nk, D], dV [nk, D]); the KV
     gradients are summed over the G query heads that share KV head g.
     """
-    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
-    B, H, S, D = q.shape
-    Hkv = k.shape[1]
+    B, H, S, D = _shape(q)
+    Hkv = _shape(k)[1]
     G = H // Hkv
     scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
     qr = _rows_arg(qrows, S)
@@ -248,8 +262,8 @@ def attn_bwd(q, k, v, dout, causal: bool, scale: float = None, qrows=None,
             need.setdefault((b, h), [False, False])[1] = True
     for (b, h), (want_q, want_kv) in sorted(need.items()):
         g = h // G
-        qh, kh = np.ascontiguousarray(q[b, h]), np.ascontiguousarray(k[b, g])
-        vh, doh = np.ascontiguousarray(v[b, g]), np.ascontiguousarray(dout[b, h])
+        qh, kh = _f64(q[b, h]), _f64(k[b, g])
+        vh, doh = _f64(v[b, g]), _f64(dout[b, h])
         nq = len(qr) if want_q else 0
         nk = len(kr) if want_kv else 0
         dq = np.zeros((max(nq, 1), D))

@@ -96,14 +96,14 @@ static double dot(const double* a, const double* b, int64_t D)
  *   LSE_i = m + ln sum_j exp(s_ij - m),  m = max_j s_ij
  *   O_i   = sum_j exp(s_ij - LSE_i) v_j
  * scratch must hold S doubles. */
-static void attend_row(const double* q, const double* k, const double* v, int64_t S,
+static void attend_row(const double* qi, const double* k, const double* v, int64_t S,
                        int64_t D, int causal, double scale, int64_t i, double* s,
                        double* o, double* lse)
 {
     int64_t n = (causal && i + 1 < S) ? i + 1 : S;
     double m = -INFINITY;
     for (int64_t j = 0; j < n; ++j) {
-        s[j] = scale * dot(q + i * D, k + j * D, D);
+        s[j] = scale * dot(qi, k + j * D, D);
         if (s[j] > m) m = s[j];
     }
     double sum = 0.0;
@@ -118,8 +118,9 @@ static void attend_row(const double* q, const double* k, const double* v, int64_
     *lse = L;
 }
 
-/* q holds the query rows named in `rows` (natural positions, row-major [*, D]);
- * k, v hold the Sk keys 0..Sk-1. Causal: query i sees keys j <= i. */
+/* q holds nrows query rows (row-major [nrows, D]); rows[r] is the natural
+ * position of q row r. k, v hold the Sk keys 0..Sk-1. Causal: the query at
+ * position i sees keys j <= i. */
 void orc_attn_fwd_head(const double* q, const double* k, const double* v, int64_t Sk,
                        int64_t D, int causal, double scale, const int64_t* rows,
                        int64_t nrows, double* o, double* lse)
@@ -129,7 +130,7 @@ void orc_attn_fwd_head(const double* q, const double* k, const double* v, int64_
         double* s = (double*)malloc(sizeof(double) * (size_t)Sk);
 #pragma omp for schedule(dynamic, 4)
         for (int64_t r = 0; r < nrows; ++r)
-            attend_row(q, k, v, Sk, D, causal, scale, rows[r], s, o + r * D, lse + r);
+            attend_row(q + r * D, k, v, Sk, D, causal, scale, rows[r], s, o + r * D, lse + r);
         free(s);
     }
 }
@@ -169,7 +170,8 @@ void orc_lse_merge(double* o_acc, double* lse_acc, const double* o_part,
 /* Ring-structured forward: per-step partials over one owner's keys, merged.  */
 /* ------------------------------------------------------------------------- */
 
-/* Query row at natural position x lives on rank i. At step t = 0..P-1 rank i
+/* q holds nrows query rows; rows[r] is the natural position of q row r.
+ * Query row at natural position x lives on rank i. At step t = 0..P-1 rank i
  * holds the key/value block of owner r = (i - t) mod P (blocks move one rank
  * forward per step). The step's partial is attention over the keys of owner r
  * that x may see; an empty set gives (0, -inf). Partials are merged in step
@@ -196,7 +198,7 @@ void orc_ring_fwd_head(const double* q, const double* k, const double* v, int64_
                 double m = -INFINITY;
                 for (int64_t j = 0; j < S; ++j) {
                     if (!rank_holds(S, P, order, r, j) || (causal && j > x)) continue;
-                    s[j] = scale * dot(q + x * D, k + j * D, D);
+                    s[j] = scale * dot(q + rr * D, k + j * D, D);
                     if (s[j] > m) m = s[j];
                 }
                 double lpart = -INFINITY;
@@ -249,7 +251,7 @@ void orc_attn_bwd_head(const double* q, const double* k, const double* v,
         for (int64_t r = 0; r < nq; ++r) {
             int64_t i = qrows[r];
             double L;
-            attend_row(q, k, v, S, D, causal, scale, i, s, oi, &L);
+            attend_row(q + i * D, k, v, S, D, causal, scale, i, s, oi, &L);
             double delta = dot(dout + i * D, oi, D);
             int64_t n = causal ? i + 1 : S;
             double* g = dq + r * D;
@@ -278,7 +280,7 @@ void orc_attn_bwd_head(const double* q, const double* k, const double* v,
         double* oi = (double*)malloc(sizeof(double) * (size_t)D);
 #pragma omp for schedule(dynamic, 16)
         for (int64_t i = i0; i < S; ++i) {
-            attend_row(q, k, v, S, D, causal, scale, i, s, oi, &lse_all[i]);
+            attend_row(q + i * D, k, v, S, D, causal, scale, i, s, oi, &lse_all[i]);
             delta_all[i] = dot(dout + i * D, oi, D);
         }
         free(oi);

@@ -1,0 +1,144 @@
+"""Blockwise ring attention with Ulysses permutes on one B200 (sm_100a).
+
+P virtual sequence-parallel ranks are simulated on one GPU; the ring's
+key/value rotation is HBM block indexing. The computation lives in librm.so
+(include/rm.h); this package is its ctypes binding (``native``) plus tensor
+conveniences that allocate outputs with PyTorch and call the C ABI.
+
+Layouts: attention tensors are [B, heads, S, D] with S in rank-major ring
+order (rank 0's S/P tokens first); ``seq_reorder`` converts from/to natural
+order. Sequence-sharded Ulysses tensors are [B, S, heads, D].
+"""
+import math
+
+from . import native
+from .native import (RM_DTYPE_BF16, RM_DTYPE_FP32, RM_HEAD_TO_SEQ,
+                     RM_NATURAL_TO_RANK_MAJOR, RM_ORDER_CONTIGUOUS, RM_ORDER_ZIGZAG,
+                     RM_RANK_MAJOR_TO_NATURAL, RM_SEQ_TO_HEAD, RMError)
+
+__all__ = ["ring_attn_fwd", "ring_attn_bwd", "lse_merge_", "ulysses_permute",
+           "ulysses_permute_qkv", "seq_reorder", "native", "RMError"]
+
+_ORDERS = {"contiguous": RM_ORDER_CONTIGUOUS, "zigzag": RM_ORDER_ZIGZAG}
+
+
+def _order(order):
+    return _ORDERS[order] if isinstance(order, str) else int(order)
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return RM_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return RM_DTYPE_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _need(t, name):
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+def ring_attn_fwd(q, k, v, P, causal=True, order="zigzag", scale=None, out=None, lse=None,
+                  stream=None):
+    """Ring attention forward. q [B,H,S,D], k/v [B,Hkv,S,D] (rank-major S).
+
+    Returns (O [B,H,S,D] in q's dtype, LSE [B,H,S] float32).
+    """
+    import torch
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n)
+    B, H, S, D = q.shape
+    Hkv = k.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    native.rm_ring_attn_fwd(q, k, v, out, lse, B, H, Hkv, S, D, P, causal, _order(order),
+                            _dtype_code(q), scale, stream)
+    return out, lse
+
+
+def ring_attn_bwd(q, k, v, o, lse, dout, P, causal=True, order="zigzag", scale=None,
+                  workspace=None, stream=None):
+    """Ring attention backward. Returns fp32 (dQ, dK, dV)."""
+    import torch
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (lse, "lse"), (dout, "dout")):
+        _need(t, n)
+    B, H, S, D = q.shape
+    Hkv = k.shape[1]
+    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=q.device)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=q.device)
+    ws_bytes = native.rm_ring_attn_bwd_workspace_size(B, H, S)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    native.rm_ring_attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace.numel(),
+                            B, H, Hkv, S, D, P, causal, _order(order), _dtype_code(q), scale,
+                            stream)
+    return dq, dk, dv
+
+
+def lse_merge_(o_acc, lse_acc, o_part, lse_part, stream=None):
+    """In-place merge of (o_part, lse_part) into (o_acc, lse_acc); fp32 [rows, D], [rows]."""
+    for t, n in ((o_acc, "o_acc"), (lse_acc, "lse_acc"), (o_part, "o_part"), (lse_part, "lse_part")):
+        _need(t, n)
+    D = o_acc.shape[-1]
+    rows = o_acc.numel() // D
+    native.rm_lse_merge(o_acc, lse_acc, o_part, lse_part, rows, D, stream)
+    return o_acc, lse_acc
+
+
+def ulysses_permute(x, U, R, direction="seq_to_head", out=None, stream=None):
+    """[B,S,Hx,D] <-> [B,Hx,S,D] (the Ulysses all-to-all on one device)."""
+    import torch
+    _need(x, "x")
+    if direction == "seq_to_head":
+        B, S, Hx, D = x.shape
+        shape, d = (B, Hx, S, D), RM_SEQ_TO_HEAD
+    else:
+        B, Hx, S, D = x.shape
+        shape, d = (B, S, Hx, D), RM_HEAD_TO_SEQ
+    if out is None:
+        out = torch.empty(shape, dtype=x.dtype, device=x.device)
+    native.rm_ulysses_permute(x, out, B, S, Hx, D, U, R, x.element_size(), d, stream)
+    return out
+
+
+def ulysses_permute_qkv(q, k, v, U, R, direction="seq_to_head", outs=None, stream=None):
+    """Fused Q/K/V Ulysses permute in one launch."""
+    import torch
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n)
+    if direction == "seq_to_head":
+        B, S, H, D = q.shape
+        Hkv = k.shape[2]
+        shapes, d = [(B, H, S, D), (B, Hkv, S, D), (B, Hkv, S, D)], RM_SEQ_TO_HEAD
+    else:
+        B, H, S, D = q.shape
+        Hkv = k.shape[1]
+        shapes, d = [(B, S, H, D), (B, S, Hkv, D), (B, S, Hkv, D)], RM_HEAD_TO_SEQ
+    if outs is None:
+        outs = [torch.empty(s, dtype=q.dtype, device=q.device) for s in shapes]
+    native.rm_ulysses_permute_qkv(q, k, v, outs[0], outs[1], outs[2], B, S, H, Hkv, D, U, R,
+                                  q.element_size(), d, stream)
+    return tuple(outs)
+
+
+def seq_reorder(x, P, order="zigzag", direction="to_rank_major", out=None, stream=None):
+    """Natural <-> rank-major token order along dim 2 of [B,H,S,D] (or [B,H,S])."""
+    import torch
+    _need(x, "x")
+    if x.dim() == 3:
+        B, H, S = x.shape
+        D = 1
+    else:
+        B, H, S, D = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    d = RM_NATURAL_TO_RANK_MAJOR if direction == "to_rank_major" else RM_RANK_MAJOR_TO_NATURAL
+    native.rm_seq_reorder(x, out, B, H, S, D, P, _order(order), d, x.element_size(), stream)
+    return out

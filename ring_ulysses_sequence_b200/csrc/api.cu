@@ -1,0 +1,252 @@
+// C ABI: argument validation, status codes, and dispatch to the kernels.
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+
+namespace rm {
+
+// Device status word: bit 0 = a bounded wait ran out. One copy per device.
+__device__ unsigned g_status_word;
+
+static thread_local int t_last_cuda_error = 0;
+static std::atomic<uint64_t> g_watchdog_ns{2000000000ull};
+
+static rm_status cuda_fail(cudaError_t e) {
+    t_last_cuda_error = static_cast<int>(e);
+    return RM_ERR_CUDA;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Status-word address and SM count of the current device, looked up once per
+// device with that device current.
+static rm_status get_ctx(cudaStream_t stream, LaunchCtx* ctx) {
+    static std::mutex mu;
+    static unsigned* word_addr[128] = {};
+    static int sms[128] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= 128) return RM_ERR_UNSUPPORTED;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!word_addr[dev]) {
+            void* p = nullptr;
+            e = cudaGetSymbolAddress(&p, g_status_word);
+            if (e != cudaSuccess) return cuda_fail(e);
+            int n = 0;
+            e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+            if (e != cudaSuccess) return cuda_fail(e);
+            sms[dev] = n;
+            word_addr[dev] = static_cast<unsigned*>(p);
+        }
+        ctx->status_word = word_addr[dev];
+        ctx->num_sms = sms[dev];
+    }
+    ctx->watchdog_ns = g_watchdog_ns.load();
+    ctx->stream = stream;
+    return RM_OK;
+}
+
+static bool valid_order(rm_order o) { return o == RM_ORDER_CONTIGUOUS || o == RM_ORDER_ZIGZAG; }
+
+// Shared shape rules of the forward and backward.
+static rm_status check_attn(const void* q, const void* k, const void* v, int B, int H, int Hkv,
+                            int S, int D, int P, rm_order order, rm_dtype dtype, float scale,
+                            int tile_q) {
+    if (B < 0 || H <= 0 || Hkv <= 0 || S < 0 || D <= 0 || P <= 0) return RM_ERR_INVALID_ARG;
+    const bool empty = B == 0 || S == 0;  // pointers of empty tensors may be null
+    if (!empty && (!q || !k || !v)) return RM_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return RM_ERR_INVALID_ARG;
+    if (!valid_order(order)) return RM_ERR_INVALID_ARG;
+    if (dtype != RM_DTYPE_BF16 && dtype != RM_DTYPE_FP32) return RM_ERR_INVALID_ARG;
+    if (!(scale > 0.0f) || !std::isfinite(scale)) return RM_ERR_INVALID_ARG;
+    if (H % Hkv != 0) return RM_ERR_INVALID_ARG;
+    if (order == RM_ORDER_ZIGZAG ? (S % (2 * P) != 0) : (S % P != 0)) return RM_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return RM_ERR_UNSUPPORTED;
+    // Tiles never straddle a chunk: the chunk must be a multiple of the tile,
+    // and (tensor-core path) a rank's block a multiple of two tiles.
+    const int64_t chunk = order == RM_ORDER_ZIGZAG ? S / (2 * P) : S / P;
+    if (chunk % tile_q != 0) return RM_ERR_UNSUPPORTED;
+    if (dtype == RM_DTYPE_BF16 && (S / P) % (2 * tile_q) != 0) return RM_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(B) * H * S >= (1ll << 31)) return RM_ERR_UNSUPPORTED;
+    return RM_OK;
+}
+
+}  // namespace rm
+
+using namespace rm;
+
+extern "C" {
+
+const char* rm_status_string(rm_status s) {
+    switch (s) {
+        case RM_OK: return "ok";
+        case RM_ERR_INVALID_ARG: return "invalid argument";
+        case RM_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case RM_ERR_CUDA: return "CUDA error";
+        case RM_ERR_TIMEOUT: return "in-kernel wait timed out";
+    }
+    return "unknown status";
+}
+
+int rm_last_cuda_error(void) { return t_last_cuda_error; }
+
+void rm_set_watchdog_ns(uint64_t ns) { g_watchdog_ns.store(ns < 1000 ? 1000 : ns); }
+
+rm_status rm_check_device_status(cudaStream_t stream) {
+    LaunchCtx ctx;
+    rm_status st = get_ctx(stream, &ctx);
+    if (st != RM_OK) return st;
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    unsigned word = 0;
+    e = cudaMemcpyFromSymbol(&word, g_status_word, sizeof(word));
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (word) {
+        const unsigned zero = 0;
+        e = cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero));
+        if (e != cudaSuccess) return cuda_fail(e);
+        return RM_ERR_TIMEOUT;
+    }
+    return RM_OK;
+}
+
+rm_status rm_watchdog_selftest(uint64_t timeout_ns, cudaStream_t stream) {
+    LaunchCtx ctx;
+    rm_status st = get_ctx(stream, &ctx);
+    if (st != RM_OK) return st;
+    ctx.watchdog_ns = timeout_ns < 1000 ? 1000 : timeout_ns;
+    cudaError_t e = launch_watchdog_selftest(ctx);
+    return e == cudaSuccess ? RM_OK : cuda_fail(e);
+}
+
+rm_status rm_ring_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                           int B, int H, int Hkv, int S, int D, int P, int causal,
+                           rm_order order, rm_dtype dtype, float scale, cudaStream_t stream) {
+    const int tile_q = dtype == RM_DTYPE_BF16 ? 128 : 64;
+    rm_status st = check_attn(q, k, v, B, H, Hkv, S, D, P, order, dtype, scale, tile_q);
+    if (st != RM_OK) return st;
+    if (B == 0 || S == 0) return RM_OK;  // empty batch or sequence: nothing to do
+    if (!o || !lse || !aligned16(o) || !aligned16(lse)) return RM_ERR_INVALID_ARG;
+    LaunchCtx ctx;
+    if ((st = get_ctx(stream, &ctx)) != RM_OK) return st;
+    AttnShape sh{B, H, Hkv, S, D, P, causal ? 1 : 0, order == RM_ORDER_ZIGZAG ? 1 : 0, scale};
+    cudaError_t e = dtype == RM_DTYPE_BF16
+                        ? launch_fwd_tc(sh, q, k, v, o, lse, ctx)
+                        : launch_fwd_fp32(sh, static_cast<const float*>(q),
+                                          static_cast<const float*>(k),
+                                          static_cast<const float*>(v), static_cast<float*>(o),
+                                          lse, ctx);
+    return e == cudaSuccess ? RM_OK : cuda_fail(e);
+}
+
+size_t rm_ring_attn_bwd_workspace_size(int B, int H, int S) {
+    if (B <= 0 || H <= 0 || S <= 0) return 0;  // empty problems need no scratch
+    const size_t delta = static_cast<size_t>(B) * H * S * sizeof(float);
+    return (delta + 255) & ~static_cast<size_t>(255);
+}
+
+rm_status rm_ring_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                           const float* lse, const void* dout, float* dq, float* dk, float* dv,
+                           void* workspace, size_t workspace_bytes, int B, int H, int Hkv,
+                           int S, int D, int P, int causal, rm_order order, rm_dtype dtype,
+                           float scale, cudaStream_t stream) {
+    rm_status st = check_attn(q, k, v, B, H, Hkv, S, D, P, order, dtype, scale, 128);
+    if (st != RM_OK) return st;
+    if (dtype != RM_DTYPE_BF16) return RM_ERR_UNSUPPORTED;
+    if (B == 0 || S == 0) return RM_OK;
+    const void* ptrs[] = {o, lse, dout, dq, dk, dv, workspace};
+    for (const void* p : ptrs)
+        if (!p || !aligned16(p)) return RM_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return RM_ERR_INVALID_ARG;
+    if (workspace_bytes < rm_ring_attn_bwd_workspace_size(B, H, S)) return RM_ERR_INVALID_ARG;
+    LaunchCtx ctx;
+    if ((st = get_ctx(stream, &ctx)) != RM_OK) return st;
+    AttnShape sh{B, H, Hkv, S, D, P, causal ? 1 : 0, order == RM_ORDER_ZIGZAG ? 1 : 0, scale};
+    cudaError_t e = launch_bwd(sh, q, k, v, o, lse, dout, dq, dk, dv,
+                               static_cast<float*>(workspace), ctx);
+    return e == cudaSuccess ? RM_OK : cuda_fail(e);
+}
+
+rm_status rm_lse_merge(float* o_acc, float* lse_acc, const float* o_part, const float* lse_part,
+                       int64_t rows, int D, cudaStream_t stream) {
+    if (rows < 0 || D <= 0) return RM_ERR_INVALID_ARG;
+    if (rows == 0) return RM_OK;
+    if (!o_acc || !lse_acc || !o_part || !lse_part) return RM_ERR_INVALID_ARG;
+    if (!aligned16(o_acc) || !aligned16(o_part) || !aligned16(lse_acc) || !aligned16(lse_part))
+        return RM_ERR_INVALID_ARG;
+    LaunchCtx ctx;
+    rm_status st = get_ctx(stream, &ctx);
+    if (st != RM_OK) return st;
+    cudaError_t e = launch_lse_merge(o_acc, lse_acc, o_part, lse_part, rows, D, ctx);
+    return e == cudaSuccess ? RM_OK : cuda_fail(e);
+}
+
+static rm_status check_permute(int B, int S, int D, int U, int R, int elem_bytes,
+                               rm_permute_dir dir) {
+    if (B < 0 || S < 0 || D <= 0 || U <= 0 || R <= 0) return RM_ERR_INVALID_ARG;
+    if (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4 && elem_bytes != 8)
+        return RM_ERR_INVALID_ARG;
+    if (dir != RM_SEQ_TO_HEAD && dir != RM_HEAD_TO_SEQ) return RM_ERR_INVALID_ARG;
+    if (S % (U * R) != 0) return RM_ERR_INVALID_ARG;
+    return RM_OK;
+}
+
+rm_status rm_ulysses_permute(const void* src, void* dst, int B, int S, int Hx, int D, int U,
+                             int R, int elem_bytes, rm_permute_dir dir, cudaStream_t stream) {
+    rm_status st = check_permute(B, S, D, U, R, elem_bytes, dir);
+    if (st != RM_OK) return st;
+    if (Hx <= 0 || Hx % U != 0) return RM_ERR_INVALID_ARG;
+    if (B == 0 || S == 0) return RM_OK;
+    if (!src || !dst || !aligned16(src) || !aligned16(dst) || src == dst) return RM_ERR_INVALID_ARG;
+    LaunchCtx ctx;
+    if ((st = get_ctx(stream, &ctx)) != RM_OK) return st;
+    PermuteTensor t{src, dst, Hx};
+    cudaError_t e = launch_ulysses_permute(&t, 1, B, S, D, elem_bytes, dir == RM_HEAD_TO_SEQ, ctx);
+    return e == cudaSuccess ? RM_OK : cuda_fail(e);
+}
+
+rm_status rm_ulysses_permute_qkv(const void* q_src, const void* k_src, const void* v_src,
+                                 void* q_dst, void* k_dst, void* v_dst, int B, int S, int H,
+                                 int Hkv, int D, int U, int R, int elem_bytes,
+                                 rm_permute_dir dir, cudaStream_t stream) {
+    rm_status st = check_permute(B, S, D, U, R, elem_bytes, dir);
+    if (st != RM_OK) return st;
+    if (H <= 0 || Hkv <= 0 || H % U != 0 || Hkv % U != 0) return RM_ERR_INVALID_ARG;
+    if (B == 0 || S == 0) return RM_OK;
+    const void* ptrs[] = {q_src, k_src, v_src, q_dst, k_dst, v_dst};
+    for (const void* p : ptrs)
+        if (!p || !aligned16(p)) return RM_ERR_INVALID_ARG;
+    LaunchCtx ctx;
+    if ((st = get_ctx(stream, &ctx)) != RM_OK) return st;
+    PermuteTensor t[3] = {{q_src, q_dst, H}, {k_src, k_dst, Hkv}, {v_src, v_dst, Hkv}};
+    cudaError_t e = launch_ulysses_permute(t, 3, B, S, D, elem_bytes, dir == RM_HEAD_TO_SEQ, ctx);
+    return e == cudaSuccess ? RM_OK : cuda_fail(e);
+}
+
+rm_status rm_seq_reorder(const void* src, void* dst, int B, int H, int S, int D, int P,
+                         rm_order order, rm_reorder_dir dir, int elem_bytes,
+                         cudaStream_t stream) {
+    if (B < 0 || H <= 0 || S < 0 || D <= 0 || P <= 0) return RM_ERR_INVALID_ARG;
+    if (!valid_order(order)) return RM_ERR_INVALID_ARG;
+    if (dir != RM_NATURAL_TO_RANK_MAJOR && dir != RM_RANK_MAJOR_TO_NATURAL)
+        return RM_ERR_INVALID_ARG;
+    if (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4 && elem_bytes != 8)
+        return RM_ERR_INVALID_ARG;
+    if (order == RM_ORDER_ZIGZAG ? (S % (2 * P) != 0) : (S % P != 0)) return RM_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(B) * H >= (1ll << 31)) return RM_ERR_UNSUPPORTED;
+    if (B == 0 || S == 0) return RM_OK;
+    if (!src || !dst || src == dst) return RM_ERR_INVALID_ARG;
+    LaunchCtx ctx;
+    rm_status st = get_ctx(stream, &ctx);
+    if (st != RM_OK) return st;
+    cudaError_t e = launch_seq_reorder(src, dst, B * H, S, D, P, order == RM_ORDER_ZIGZAG,
+                                       dir == RM_RANK_MAJOR_TO_NATURAL, elem_bytes, ctx);
+    return e == cudaSuccess ? RM_OK : cuda_fail(e);
+}
+
+}  // extern "C"

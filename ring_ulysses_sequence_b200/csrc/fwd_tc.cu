@@ -1,0 +1,488 @@
+// Ring attention forward, bf16 in / fp32 accumulate, on the sm_100a tensor
+// cores (tcgen05.mma with TMEM accumulators, TMA-staged tiles).
+//
+// What it computes ("DeDLOC Guide: Decentralized Long-Context Attention",
+// Step 3 local step and section 3 online-softmax merge; "Sequence Parallelism
+// III: Ring Attention ...", duoan.github.io): every query tile of virtual rank
+// i keeps its block fixed and visits the key/value block of owner
+// r = (i - t) mod P at ring step t = 0..P-1. Each visit is a flash tile pass
+// S = Q K^T, causal mask on global positions, online softmax, O += P V. The
+// running (m, l, O) simply continues across step boundaries, which is exactly
+// the alpha/beta merge of the steps' (O, LSE) partials, done in registers and
+// TMEM. Tiles the causal mask hides completely are never computed ("DeDLOC
+// Guide", Best Practices, Causal Mask Handling).
+//
+// Block structure (persistent, one CTA per SM, 320 threads):
+//   warps 0-3  softmax warpgroup for query tile 0, warps 4-7 for tile 1
+//              (thread = one query row = one TMEM lane); they also write O/LSE
+//   warp 8     MMA issuer (one thread)
+//   warp 9     TMA producer (one thread)
+// The two query tiles share every K/V tile: they are two heads of one GQA
+// group at the same slots, or (odd group size) two consecutive 128-slot tiles
+// of one head within one rank.
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [384,384+D).
+// P (bf16) overwrites the first 64 columns of its S tile and is the TMEM
+// A-operand of the PV product. Issue order per key tile j:
+//   PV0_j, QK0_{j+1}, PV1_j, QK1_{j+1}
+// so the tensor pipe runs one tile's products while the other tile's softmax
+// runs. O is rescaled only when a row maximum grows by more than 2^8 (in exp2
+// units); the sum l uses the same reference maximum, so the result is exact.
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tmap.h"
+
+namespace rm {
+
+namespace {
+
+constexpr int kBM = 128;        // query rows per tile (UMMA M)
+constexpr int kBN = 128;        // keys per tile (UMMA N of QK^T, K of PV)
+constexpr int kStages = 4;      // K/V ring in shared memory (one tile per stage)
+constexpr int kThreads = 320;
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp = 9;
+constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest stale-max factor
+
+template <int D>
+struct Cfg {
+    static constexpr int kTileBytes = kBM * D * 2;  // one Q, K or V tile
+    static constexpr int kBoxes = D / 64;           // 128-byte swizzle boxes along D
+    static constexpr int kBoxBytes = kBM * 128;     // 16 KB
+    static constexpr int kQOff = 0;
+    static constexpr int kKVOff = 2 * kTileBytes;
+    static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
+    static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + barriers + alignment slack
+};
+
+struct TcArgs {
+    CUtensorMap tm_q, tm_k, tm_v;
+    void* o;
+    float* lse;
+    unsigned* status;
+    unsigned long long timeout_ns;
+    int H, Hkv, S, P, causal, G;
+    int head_pair;     // 1: tiles are heads (h, h+1) at one slot; 0: one head, slots s, s+128
+    int n_units;       // query units per head unit
+    int n_head_units;  // B * (head_pair ? H / 2 : H)
+    int n_items;
+    float scale, scale_log2;
+    RingLayout lay;
+};
+
+struct Item {
+    int b, h0, h1, g, slot0, slot1, pos0, pos1, rank;
+};
+
+// Work item w -> two query tiles. Items are ordered by the natural position of
+// their queries, latest first when causal (the most key tiles first), with the
+// heads of one position adjacent so that concurrent CTAs share K/V in L2.
+__device__ __forceinline__ Item decode_item(const TcArgs& a, int w) {
+    Item it;
+    const int unit_rank = w / a.n_head_units;
+    const int hu = w - unit_rank * a.n_head_units;
+    const int heads_per_b = a.head_pair ? a.H / 2 : a.H;
+    it.b = hu / heads_per_b;
+    const int hh = hu - it.b * heads_per_b;
+    it.h0 = a.head_pair ? 2 * hh : hh;
+    it.h1 = a.head_pair ? it.h0 + 1 : it.h0;
+    it.g = it.h0 / a.G;
+    const int U = a.head_pair ? kBM : 2 * kBM;
+    const int nu = a.causal ? a.n_units - 1 - unit_rank : unit_rank;
+    int slot;
+    if (!a.lay.zigzag || a.lay.c % U == 0)
+        slot = a.lay.slot_of_pos(nu * U);  // the unit is contiguous in slots too
+    else
+        slot = nu * U;                     // chunk of one tile: take slot order
+    it.slot0 = slot;
+    it.slot1 = a.head_pair ? slot : slot + kBM;
+    it.pos0 = a.lay.pos_of_slot(it.slot0);
+    it.pos1 = a.lay.pos_of_slot(it.slot1);
+    it.rank = slot / a.lay.L;
+    return it;
+}
+
+// Causal class of a (query tile, key tile) pair; both start on multiples of
+// 128 in natural positions (chunks are multiples of 128 tokens).
+enum : int { kSkip = 0, kDiag = 1, kFull = 2 };
+__device__ __forceinline__ int tile_class(int causal, int qpos, int kpos) {
+    if (!causal) return kFull;
+    return kpos > qpos ? kSkip : (kpos == qpos ? kDiag : kFull);
+}
+
+// Key tiles of an item in ring order: step t visits owner (rank - t) mod P.
+struct KvIter {
+    RingLayout lay;
+    int rank, causal, pos0, pos1, t, u, ntile;
+    __device__ __forceinline__ KvIter(const TcArgs& a, const Item& it)
+        : lay(a.lay), rank(it.rank), causal(a.causal), pos0(it.pos0), pos1(it.pos1), t(0), u(0),
+          ntile(a.lay.L / kBN) {}
+    __device__ __forceinline__ bool next(int& kslot, int& c0, int& c1) {
+        while (t < lay.P) {
+            const int ks = lay.owner(rank, t) * lay.L + u * kBN;
+            if (++u == ntile) { u = 0; ++t; }
+            const int kp = lay.pos_of_slot(ks);
+            c0 = tile_class(causal, pos0, kp);
+            c1 = tile_class(causal, pos1, kp);
+            if (c0 != kSkip || c1 != kSkip) { kslot = ks; return true; }
+        }
+        return false;
+    }
+};
+
+struct Bars {
+    uint64_t q_full, q_empty, drain;
+    uint64_t kv_full[kStages], kv_empty[kStages];
+    uint64_t s_full[2], p_full[2], o_full[2];
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+template <int D>
+__device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_smem, uint32_t k_smem) {
+    constexpr uint32_t idesc = umma_idesc_bf16(kBM, kBN, 0, 0);
+#pragma unroll
+    for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = (k >> 2) * Cfg<D>::kBoxBytes + (k & 3) * 32;
+        umma_ss(tmem_s, umma_desc_sw128(q_smem + off, 16, 1024),
+                umma_desc_sw128(k_smem + off, 16, 1024), idesc, k > 0 ? 1u : 0u);
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_smem,
+                                         bool accumulate) {
+    constexpr uint32_t idesc = umma_idesc_bf16(kBM, D, 0, 1);
+#pragma unroll
+    for (int k = 0; k < kBN / 16; ++k)
+        umma_ts(tmem_o, tmem_p + 8 * k,
+                umma_desc_sw128(v_smem + k * 2048, Cfg<D>::kBoxBytes, 1024), idesc,
+                (accumulate || k > 0) ? 1u : 0u);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_constant__ TcArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    Bars& bars = *reinterpret_cast<Bars*>(smem + Cfg<D>::kBarOff);
+    const uint32_t q_smem = smem_u32(smem + Cfg<D>::kQOff);
+    const uint32_t kv_smem = smem_u32(smem + Cfg<D>::kKVOff);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        bars.abort_flag = 0;
+        mbar_init(smem_u32(&bars.q_full), 1);
+        mbar_init(smem_u32(&bars.q_empty), 1);
+        mbar_init(smem_u32(&bars.drain), 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(smem_u32(&bars.kv_full[s]), 1);
+            mbar_init(smem_u32(&bars.kv_empty[s]), 1);
+        }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(smem_u32(&bars.s_full[x]), 1);
+            mbar_init(smem_u32(&bars.p_full[x]), 128);
+            mbar_init(smem_u32(&bars.o_full[x]), 1);
+        }
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&bars.tmem_base), 512);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars.tmem_base;
+    const Watchdog wd{a.status, &bars.abort_flag, a.timeout_ns};
+
+    if (warp == kLoadWarp) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tmap(&a.tm_q);
+            prefetch_tmap(&a.tm_k);
+            prefetch_tmap(&a.tm_v);
+            uint32_t q_iter = 0, kv_iter = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x) {
+                const Item it = decode_item(a, w);
+                if (q_iter > 0) ok = mbar_wait(smem_u32(&bars.q_empty), (q_iter - 1) & 1, wd);
+                if (!ok) break;
+                ++q_iter;
+                mbar_arrive_expect_tx(smem_u32(&bars.q_full), 2 * Cfg<D>::kTileBytes);
+                for (int x = 0; x < 2; ++x) {
+                    const int row = ((it.b * a.H) + (x ? it.h1 : it.h0)) * a.S + (x ? it.slot1 : it.slot0);
+                    for (int bx = 0; bx < Cfg<D>::kBoxes; ++bx)
+                        tma_load_2d(q_smem + x * Cfg<D>::kTileBytes + bx * Cfg<D>::kBoxBytes, &a.tm_q,
+                                    bx * 64, row, smem_u32(&bars.q_full));
+                }
+                KvIter kv(a, it);
+                int kslot, c0, c1;
+                while (ok && kv.next(kslot, c0, c1)) {
+                    const int row = (it.b * a.Hkv + it.g) * a.S + kslot;
+                    for (int which = 0; which < 2 && ok; ++which) {  // K then V
+                        const int st = kv_iter % kStages;
+                        const uint32_t use = kv_iter / kStages;
+                        if (use > 0) ok = mbar_wait(smem_u32(&bars.kv_empty[st]), (use - 1) & 1, wd);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(smem_u32(&bars.kv_full[st]), Cfg<D>::kTileBytes);
+                        for (int bx = 0; bx < Cfg<D>::kBoxes; ++bx)
+                            tma_load_2d(kv_smem + st * Cfg<D>::kTileBytes + bx * Cfg<D>::kBoxBytes,
+                                        which ? &a.tm_v : &a.tm_k, bx * 64, row,
+                                        smem_u32(&bars.kv_full[st]));
+                        ++kv_iter;
+                    }
+                }
+            }
+            if (!ok) {
+                // Let the copies already issued land before the CTA exits; the
+                // abort flag is up, so these waits use a watchdog of their own.
+                volatile int no_abort = 0;
+                const Watchdog w2{a.status, &no_abort, a.timeout_ns};
+                for (uint32_t i = kv_iter > kStages ? kv_iter - kStages : 0; i < kv_iter; ++i)
+                    (void)mbar_wait(smem_u32(&bars.kv_full[i % kStages]), (i / kStages) & 1, w2);
+                if (q_iter > 0) (void)mbar_wait(smem_u32(&bars.q_full), (q_iter - 1) & 1, w2);
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t tS[2] = {tmem, tmem + 128};
+            const uint32_t tO[2] = {tmem + 256, tmem + 384};
+            uint32_t q_iter = 0, kv_iter = 0, p_cnt[2] = {0, 0};
+            bool ok = true;
+            for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x) {
+                const Item it = decode_item(a, w);
+                int n = 0;
+                {
+                    KvIter kv(a, it);
+                    int ks, c0, c1;
+                    while (kv.next(ks, c0, c1)) ++n;
+                }
+                ok = mbar_wait(smem_u32(&bars.q_full), q_iter & 1, wd);
+                if (!ok) break;
+                ++q_iter;
+                // prologue: S_x = Q_x K_0^T
+                uint32_t stK = kv_iter % kStages;
+                ok = mbar_wait(smem_u32(&bars.kv_full[stK]), (kv_iter / kStages) & 1, wd);
+                if (!ok) break;
+                ++kv_iter;
+                tc_fence_after();
+                issue_qk<D>(tS[0], q_smem, kv_smem + stK * Cfg<D>::kTileBytes);
+                umma_commit(smem_u32(&bars.s_full[0]));
+                issue_qk<D>(tS[1], q_smem + Cfg<D>::kTileBytes, kv_smem + stK * Cfg<D>::kTileBytes);
+                umma_commit(smem_u32(&bars.s_full[1]));
+                umma_commit(smem_u32(&bars.kv_empty[stK]));
+                if (n == 1) umma_commit(smem_u32(&bars.q_empty));
+                for (int j = 0; j < n && ok; ++j) {
+                    const uint32_t stV = kv_iter % kStages;
+                    ok = mbar_wait(smem_u32(&bars.kv_full[stV]), (kv_iter / kStages) & 1, wd);
+                    if (!ok) break;
+                    ++kv_iter;
+                    const uint32_t v_addr = kv_smem + stV * Cfg<D>::kTileBytes;
+                    ok = mbar_wait(smem_u32(&bars.p_full[0]), (p_cnt[0]++) & 1, wd);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv<D>(tO[0], tS[0], v_addr, j > 0);
+                    if (j == n - 1) umma_commit(smem_u32(&bars.o_full[0]));
+                    const bool more = j + 1 < n;
+                    if (more) {
+                        stK = kv_iter % kStages;
+                        ok = mbar_wait(smem_u32(&bars.kv_full[stK]), (kv_iter / kStages) & 1, wd);
+                        if (!ok) break;
+                        ++kv_iter;
+                        tc_fence_after();
+                        issue_qk<D>(tS[0], q_smem, kv_smem + stK * Cfg<D>::kTileBytes);
+                        umma_commit(smem_u32(&bars.s_full[0]));
+                    }
+                    ok = mbar_wait(smem_u32(&bars.p_full[1]), (p_cnt[1]++) & 1, wd);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv<D>(tO[1], tS[1], v_addr, j > 0);
+                    umma_commit(smem_u32(&bars.kv_empty[stV]));
+                    if (j == n - 1) umma_commit(smem_u32(&bars.o_full[1]));
+                    if (more) {
+                        issue_qk<D>(tS[1], q_smem + Cfg<D>::kTileBytes,
+                                    kv_smem + stK * Cfg<D>::kTileBytes);
+                        umma_commit(smem_u32(&bars.s_full[1]));
+                        umma_commit(smem_u32(&bars.kv_empty[stK]));
+                        if (j + 1 == n - 1) umma_commit(smem_u32(&bars.q_empty));
+                    }
+                }
+            }
+            // Every product issued must finish before TMEM is released.
+            umma_commit(smem_u32(&bars.drain));
+            volatile int no_abort = 0;
+            const Watchdog w2{a.status, &no_abort, a.timeout_ns};
+            (void)mbar_wait(smem_u32(&bars.drain), 0, w2);
+        }
+    } else {
+        // ------------------------------------------------------------ softmax
+        const int x = warp >> 2;                    // query tile of this warpgroup
+        const int quarter = warp & 3;               // TMEM lane quarter
+        const int r = quarter * 32 + lane;          // query row in the tile
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        const uint32_t tS = tmem + lane_off + x * 128;
+        const uint32_t tO = tmem + lane_off + 256 + x * 128;
+        const float sl2 = a.scale_log2;
+        uint32_t s_cnt = 0, o_cnt = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x) {
+            const Item it = decode_item(a, w);
+            float m = -INFINITY, l = 0.f;
+            KvIter kv(a, it);
+            int kslot, c0, c1, j = 0;
+            while (ok && kv.next(kslot, c0, c1)) {
+                const int cls = x ? c1 : c0;
+                ok = mbar_wait(smem_u32(&bars.s_full[x]), (s_cnt++) & 1, wd);
+                if (!ok) break;
+                tc_fence_after();
+                if (cls == kSkip) {
+                    uint32_t z[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) z[c] = 0u;
+                    tmem_st32(tS, z);
+                    tmem_st32(tS + 32, z);
+                } else {
+                    uint32_t raw[64];
+                    float s[128];
+                    tmem_ld64(tS, raw);
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(raw[c]);
+                    tmem_ld64(tS + 64, raw);
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) s[64 + c] = __uint_as_float(raw[c]);
+                    if (cls == kDiag) {
+#pragma unroll
+                        for (int c = 0; c < 128; ++c)
+                            if (c > r) s[c] = -INFINITY;
+                    }
+                    float mx = s[0];
+#pragma unroll
+                    for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+                    const float m_new = fmaxf(m, mx);
+                    float alpha = 1.f;
+                    bool rescale_o = false;
+                    if ((m_new - m) * sl2 > kRescaleThreshold) {
+                        alpha = ex2_approx((m - m_new) * sl2);  // 0 when m = -inf
+                        l *= alpha;
+                        m = m_new;
+                        rescale_o = j > 0;
+                    }
+                    const float neg = -m * sl2;  // m is finite after a visible tile
+                    float rs = 0.f;
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int c = 0; c < 64; c += 2) {
+                        const float p0 = ex2_approx(fmaf(s[c], sl2, neg));
+                        const float p1 = ex2_approx(fmaf(s[c + 1], sl2, neg));
+                        rs += p0 + p1;
+                        pk[c >> 1] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st32(tS, pk);
+#pragma unroll
+                    for (int c = 64; c < 128; c += 2) {
+                        const float p0 = ex2_approx(fmaf(s[c], sl2, neg));
+                        const float p1 = ex2_approx(fmaf(s[c + 1], sl2, neg));
+                        rs += p0 + p1;
+                        pk[(c - 64) >> 1] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st32(tS + 32, pk);
+                    l += rs;
+                    if (__any_sync(0xffffffffu, rescale_o)) {
+                        const float f = rescale_o ? alpha : 1.f;
+#pragma unroll 1
+                        for (int cc = 0; cc < D; cc += 32) {
+                            uint32_t ov[32];
+                            tmem_ld32(tO + cc, ov);
+#pragma unroll
+                            for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * f);
+                            tmem_st32(tO + cc, ov);
+                        }
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(smem_u32(&bars.p_full[x]));
+                ++j;
+            }
+            if (!ok) break;
+            // epilogue: O / l -> bf16, LSE = m * scale + ln l
+            ok = mbar_wait(smem_u32(&bars.o_full[x]), (o_cnt++) & 1, wd);
+            if (!ok) break;
+            tc_fence_after();
+            const int h = x ? it.h1 : it.h0;
+            const int64_t orow = (static_cast<int64_t>(it.b) * a.H + h) * a.S + (x ? it.slot1 : it.slot0) + r;
+            const float inv = l > 0.f ? 1.0f / l : 0.f;
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + orow * D);
+#pragma unroll 1
+            for (int cc = 0; cc < D; cc += 32) {
+                uint32_t ov[32];
+                tmem_ld32(tO + cc, ov);
+                uint32_t pk[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    pk[c] = pack_bf16x2(__uint_as_float(ov[2 * c]) * inv, __uint_as_float(ov[2 * c + 1]) * inv);
+#pragma unroll
+                for (int v4 = 0; v4 < 4; ++v4)
+                    dst[cc / 8 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+            }
+            a.lse[orow] = l > 0.f ? m * a.scale + logf(l) : -INFINITY;
+        }
+    }
+
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_tc(const AttnShape& sh, const void* q, const void* k, const void* v,
+                          void* o, float* lse, const LaunchCtx& ctx) {
+    TcArgs a{};
+    cudaError_t e;
+    const uint64_t qrows = static_cast<uint64_t>(sh.B) * sh.H * sh.S;
+    const uint64_t kvrows = static_cast<uint64_t>(sh.B) * sh.Hkv * sh.S;
+    if ((e = make_tmap_bf16_rows(&a.tm_q, q, qrows, sh.D, kBM, 64)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16_rows(&a.tm_k, k, kvrows, sh.D, kBN, 64)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16_rows(&a.tm_v, v, kvrows, sh.D, kBN, 64)) != cudaSuccess) return e;
+    a.o = o;
+    a.lse = lse;
+    a.status = ctx.status_word;
+    a.timeout_ns = ctx.watchdog_ns;
+    a.H = sh.H;
+    a.Hkv = sh.Hkv;
+    a.S = sh.S;
+    a.P = sh.P;
+    a.causal = sh.causal;
+    a.G = sh.H / sh.Hkv;
+    a.head_pair = (a.G % 2 == 0) ? 1 : 0;
+    a.n_units = a.head_pair ? sh.S / kBM : sh.S / (2 * kBM);
+    a.n_head_units = sh.B * (a.head_pair ? sh.H / 2 : sh.H);
+    a.n_items = a.n_units * a.n_head_units;
+    a.scale = sh.scale;
+    a.scale_log2 = sh.scale * 1.4426950408889634f;
+    a.lay = RingLayout{sh.S, sh.P, sh.S / sh.P, sh.zigzag ? sh.S / (2 * sh.P) : sh.S / sh.P,
+                       sh.zigzag};
+    const int grid = std::min(a.n_items, ctx.num_sms);
+    if (sh.D == 64) {
+        constexpr int smem = Cfg<64>::kSmemBytes;
+        if ((e = cudaFuncSetAttribute(ring_fwd_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      smem)) != cudaSuccess)
+            return e;
+        ring_fwd_tc_kernel<64><<<grid, kThreads, smem, ctx.stream>>>(a);
+    } else {
+        constexpr int smem = Cfg<128>::kSmemBytes;
+        if ((e = cudaFuncSetAttribute(ring_fwd_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      smem)) != cudaSuccess)
+            return e;
+        ring_fwd_tc_kernel<128><<<grid, kThreads, smem, ctx.stream>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace rm

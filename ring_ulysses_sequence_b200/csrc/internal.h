@@ -1,0 +1,49 @@
+// Host-side interfaces between the C ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "rm.h"
+
+namespace rm {
+
+// Per-launch context: device status word, watchdog limit, device properties.
+struct LaunchCtx {
+    unsigned* status_word;   // device address of the status word
+    uint64_t watchdog_ns;
+    int num_sms;
+    cudaStream_t stream;
+};
+
+struct AttnShape {
+    int B, H, Hkv, S, D, P, causal, zigzag;
+    float scale;
+};
+
+// Forward, bf16, tcgen05 tensor cores (fwd_tc.cu).
+cudaError_t launch_fwd_tc(const AttnShape& sh, const void* q, const void* k, const void* v,
+                          void* o, float* lse, const LaunchCtx& ctx);
+// Forward, fp32 FMA path (fwd_simt.cu).
+cudaError_t launch_fwd_fp32(const AttnShape& sh, const float* q, const float* k, const float* v,
+                            float* o, float* lse, const LaunchCtx& ctx);
+// Backward, bf16 (bwd.cu). workspace holds Delta [B, H, S] fp32.
+cudaError_t launch_bwd(const AttnShape& sh, const void* q, const void* k, const void* v,
+                       const void* o, const float* lse, const void* dout, float* dq, float* dk,
+                       float* dv, float* delta, const LaunchCtx& ctx);
+
+// Layout kernels (layout.cu).
+struct PermuteTensor {
+    const void* src;
+    void* dst;
+    int heads;
+};
+cudaError_t launch_ulysses_permute(const PermuteTensor* t, int ntensors, int B, int S, int D,
+                                   int elem_bytes, int head_to_seq, const LaunchCtx& ctx);
+cudaError_t launch_seq_reorder(const void* src, void* dst, int BH, int S, int D, int P,
+                               int zigzag, int to_natural, int elem_bytes, const LaunchCtx& ctx);
+cudaError_t launch_lse_merge(float* o_acc, float* lse_acc, const float* o_part,
+                             const float* lse_part, int64_t rows, int D, const LaunchCtx& ctx);
+cudaError_t launch_watchdog_selftest(const LaunchCtx& ctx);
+
+}  // namespace rm

@@ -1,0 +1,123 @@
+"""CPU checks of the C ABI: the library loads, exports every symbol the header
+declares, and its host-side validation rejects bad arguments before touching
+the GPU (no compute calls are made here)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rm.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from ring_ulysses_sequence_b200 import build, native
+    build.build()
+    return native.lib()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^RM_API\s+[\w\s\*]*?\b(rm_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_path():
+    fns = header_functions()
+    for name in ("rm_ring_attn_fwd", "rm_ring_attn_bwd", "rm_ring_attn_bwd_workspace_size",
+                 "rm_lse_merge", "rm_ulysses_permute", "rm_ulysses_permute_qkv",
+                 "rm_seq_reorder", "rm_check_device_status", "rm_status_string"):
+        assert name in fns
+
+
+def test_library_exports_every_header_symbol(lib):
+    from ring_ulysses_sequence_b200 import native
+    out = subprocess.run(["nm", "-D", "--defined-only", native.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\b(rm_\w+)\b", out))
+    for name in header_functions():
+        assert name in exported, name
+        assert getattr(lib, name) is not None
+    # and the binding declares exactly the header's functions
+    assert sorted(native.SIGNATURES) == header_functions()
+
+
+def test_status_strings(lib):
+    from ring_ulysses_sequence_b200 import native
+    assert native.rm_status_string(0) == "ok"
+    assert "timed out" in native.rm_status_string(4)
+    assert native.rm_status_string(99) == "unknown status"
+
+
+def test_workspace_size(lib):
+    from ring_ulysses_sequence_b200 import native
+    assert native.rm_ring_attn_bwd_workspace_size(1, 2, 1024) == 2 * 1024 * 4
+    assert native.rm_ring_attn_bwd_workspace_size(1, 1, 3) == 256  # rounded to 256 B
+    assert native.rm_ring_attn_bwd_workspace_size(0, 2, 1024) == 0
+
+
+A = 1 << 20  # a fake, 16-byte aligned "device address" (never dereferenced)
+
+
+def fwd(lib, **kw):
+    args = dict(q=A, k=A, v=A, o=A, lse=A, B=1, H=4, Hkv=2, S=1024, D=128, P=4, causal=1,
+                order=1, dtype=0, scale=0.088, stream=None)
+    args.update(kw)
+    return lib.rm_ring_attn_fwd(args["q"], args["k"], args["v"], args["o"], args["lse"],
+                                args["B"], args["H"], args["Hkv"], args["S"], args["D"],
+                                args["P"], args["causal"], args["order"], args["dtype"],
+                                args["scale"], args["stream"])
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=None), 1), (dict(lse=None), 1), (dict(k=A + 8), 1),          # null / misaligned
+    (dict(H=3, Hkv=2), 1), (dict(B=-1), 1), (dict(P=0), 1), (dict(B=0), 0), (dict(S=0), 0),
+    (dict(order=7), 1), (dict(dtype=5), 1), (dict(scale=0.0), 1), (dict(scale=float("nan")), 1),
+    (dict(S=1004), 1),                                                   # not a multiple of 2P
+    (dict(D=96), 2), (dict(S=1024, P=8), 2),                             # chunk 64 < 128 tile
+    (dict(order=0, S=768, P=4), 2),                                      # contiguous block 192
+])
+def test_forward_validation(lib, kw, expect):
+    assert fwd(lib, **kw) == expect
+
+
+def test_backward_validation(lib):
+    base = [A] * 10 + [1 << 16, 1, 4, 2, 1024, 128, 4, 1, 1, 0, 0.088, None]
+    assert lib.rm_ring_attn_bwd(*base[:9], None, *base[10:]) == 1          # no workspace
+    small = list(base)
+    small[10] = 64
+    assert lib.rm_ring_attn_bwd(*small) == 1                               # too small
+    fp32 = list(base)
+    fp32[19] = 1
+    assert lib.rm_ring_attn_bwd(*fp32) == 2                                # fp32 unsupported
+    mis = list(base)
+    mis[9] = A + 16                                                        # workspace not 256-aligned
+    assert lib.rm_ring_attn_bwd(*mis) == 1
+
+
+def test_layout_validation(lib):
+    # permute: heads not divisible by U, bad element size, aliasing, bad direction
+    assert lib.rm_ulysses_permute(A, A * 2, 1, 1024, 6, 128, 4, 2, 2, 0, None) == 1
+    assert lib.rm_ulysses_permute(A, A * 2, 1, 1024, 8, 128, 4, 2, 3, 0, None) == 1
+    assert lib.rm_ulysses_permute(A, A, 1, 1024, 8, 128, 4, 2, 2, 0, None) == 1
+    assert lib.rm_ulysses_permute(A, A * 2, 1, 1024, 8, 128, 4, 2, 2, 9, None) == 1
+    assert lib.rm_ulysses_permute(A, A * 2, 1, 1004, 8, 128, 4, 2, 2, 0, None) == 1  # S % (U R)
+    # fused: KV heads must be divisible by U as well (Ulysses is capped by KV heads)
+    assert lib.rm_ulysses_permute_qkv(A, A, A, A, A, A, 1, 1024, 32, 2, 128, 4, 2, 2, 0, None) == 1
+    # reorder
+    assert lib.rm_seq_reorder(A, A * 2, 1, 2, 1000, 4, 8, 1, 0, 2, None) == 1  # S % 2P
+    assert lib.rm_seq_reorder(A, A, 1, 2, 1024, 4, 8, 1, 0, 2, None) == 1      # in place
+    assert lib.rm_seq_reorder(A, A * 2, 1, 2, 1024, 4, 8, 3, 0, 2, None) == 1  # bad order
+    # merge
+    assert lib.rm_lse_merge(A, A, A, A, -1, 4, None) == 1
+    assert lib.rm_lse_merge(None, None, None, None, 0, 4, None) == 0            # nothing to do
+    assert lib.rm_lse_merge(A, A, A + 4, A, 10, 4, None) == 1                   # misaligned
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_valid_call_without_gpu_reports_cuda_error(lib):
+    assert fwd(lib) == 3
+    assert lib.rm_last_cuda_error() != 0
