@@ -1,0 +1,471 @@
+#!/usr/bin/env python
+"""Benchmark of the ring attention hot path on B200.
+
+Headline: causal-adjusted attention TFLOPS of the ring forward on the Llama-3-8B
+layer shape at 32k tokens (B=1, 32 query heads over 8 KV heads, D=128, P=8
+virtual ranks in zigzag order, causal, bf16 in / fp32 accumulate), as a
+fraction of the measured dense BF16 peak. One step = one forward launch over
+one batch of synthetic input already resident in HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs its own replica (weak scaling, no exchange: the
+ring is simulated on each GPU); the time is the max over ranks. Also reported:
+e2e (host buffers, copies inside the timed region), the roofline of the
+forward kernel, the CPU oracle as a baseline, sampled SM clocks, and the
+other hot-path kernels (Ulysses permute, backward) as extra entries.
+`--impl reference` times the fp64 CPU oracle on bounded samples of the same
+workload and prints the same line with "impl": "reference".
+"""
+import argparse
+import faulthandler
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+faulthandler.enable()
+
+METRIC = "causal-adj attention TFLOPS, % of B200 BF16 peak (S=32k GQA ring fwd)"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--only", choices=["all", "fwd", "permute", "bwd"], default="all",
+                   help="restrict to one kernel (used for profiling runs)")
+    p.add_argument("--skip-cpu", action="store_true", help="skip the CPU oracle baseline")
+    p.add_argument("--skip-e2e", action="store_true")
+    args = p.parse_args()
+    if args.warmup < 3 and args.only == "all":
+        p.error("at least 3 warm-up steps")
+    return args
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_digest(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(summary_name, sources):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of the kernel (else None)."""
+    path = os.path.join(ROOT, "profiles", summary_name)
+    try:
+        kv = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line and not line.startswith(" "):
+                    k, v = line.split(":", 1)
+                    kv[k.strip()] = v.strip()
+        if kv.get("source_sha256") != source_digest(sources):
+            return None
+        return float(kv["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
+
+    def __init__(self, device_index, period_s=0.05):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._t = None
+        self.handle = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            want = (getattr(props, "pci_domain_id", None), getattr(props, "pci_bus_id", None),
+                    getattr(props, "pci_device_id", None))
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                info = pynvml.nvmlDeviceGetPciInfo(h)
+                if (int(info.domain), int(info.bus), int(info.device)) == want:
+                    self.handle = h
+                    break
+            if self.handle is not None:
+                self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+                self.nvml = pynvml
+        except Exception:
+            self.handle = None
+
+    def _run(self):
+        nv = self.nvml
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM))
+                bits = int(get_reasons(self.handle))
+                for b, name in self.REASONS.items():
+                    if bits & b and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.handle is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def time_on_stream(fn, steps, stream):
+    """Device time (ms) of `steps` calls of fn, with CUDA events on `stream`."""
+    import torch
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        fn()
+    end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end)
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline and reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(w, nrows_per_head, seed):
+    """Times the fp64 oracle on nrows_per_head seeded query rows of every head
+    of workload w. Returns (seconds, algorithmic FLOPs of the sample, threads)."""
+    import numpy as np
+    import oracle
+    from ring_ulysses_sequence_b200.synth import make_inputs
+    if not hasattr(oracle_sample, "_cache"):
+        oracle_sample._cache = {}
+    if w.name not in oracle_sample._cache:
+        q, k, v = make_inputs(w, with_dout=False)
+        oracle_sample._cache[w.name] = (q.float(), k.float(), v.float())
+    q, k, v = oracle_sample._cache[w.name]
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(w.S, size=nrows_per_head, replace=False))
+    t0 = time.perf_counter()
+    oracle.attn_fwd(q, k, v, w.causal, rows=rows)
+    dt = time.perf_counter() - t0
+    keys = (rows + 1) if w.causal else np.full(len(rows), w.S)
+    flops = float(4.0 * w.D * keys.sum() * w.B * w.H)
+    return dt, flops, oracle.num_threads()
+
+
+def calibrate_rows(w, target_s, seed=0, lo=16, hi=4096):
+    """Rows per head that make one oracle sample take about target_s seconds
+    (two-point fit: the per-call fixed cost is separated from the per-row cost)."""
+    t_lo, _, _ = oracle_sample(w, lo, seed)
+    t_hi, _, _ = oracle_sample(w, 4 * lo, seed + 1)
+    per_row = max((t_hi - t_lo) / (3 * lo), 1e-6)
+    fixed = max(t_lo - lo * per_row, 0.0)
+    return int(max(lo, min(hi, (target_s - fixed) / per_row)))
+
+
+def cpu_baseline(w, target_s=15.0):
+    n = calibrate_rows(w, target_s)
+    dt, flops, threads = oracle_sample(w, n, seed=12345)
+    return {"value": flops / dt / 1e12, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+            "sample": f"{n} seeded query rows of each of the {w.B * w.H} heads "
+                      f"(all their visible keys), fp64, {dt:.1f} s"}
+
+
+def run_reference(args):
+    from ring_ulysses_sequence_b200 import multi
+    from ring_ulysses_sequence_b200.synth import BENCH_WORKLOAD, WORKLOADS
+    rank, world, _ = multi.env_ranks()
+    if rank != 0:
+        return
+    w = WORKLOADS[BENCH_WORKLOAD]
+    per_step = max(0.3, min(10.0, 150.0 / (args.steps + args.warmup)))
+    n = calibrate_rows(w, per_step)
+    for i in range(args.warmup):
+        oracle_sample(w, n, seed=i)
+    tot_s, tot_f, threads = 0.0, 0.0, 1
+    for i in range(args.steps):
+        dt, fl, threads = oracle_sample(w, n, seed=1000 + i)
+        tot_s += dt
+        tot_f += fl
+    value = tot_f / tot_s / 1e12
+    sample = (f"per step {n} seeded query rows of each of the {w.B * w.H} heads "
+              f"(all their visible keys), fp64 oracle")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot_s / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w):
+    return {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.Hkv, "S": w.S, "D": w.D, "P": w.P,
+            "order": w.order, "causal": w.causal, "global_batch": w.B, "seq_len": w.S,
+            "parallelism": f"ring P={w.P} simulated per GPU"}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def bench_forward(w, args, dev, stream):
+    import torch
+    import ring_ulysses_sequence_b200 as rm
+    from ring_ulysses_sequence_b200 import multi
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed)
+    q = (torch.randn((w.B, w.H, w.S, w.D), generator=g, device=dev) * w.input_scale).to(w.dtype)
+    k = (torch.randn((w.B, w.Hkv, w.S, w.D), generator=g, device=dev) * w.input_scale).to(w.dtype)
+    v = (torch.randn((w.B, w.Hkv, w.S, w.D), generator=g, device=dev) * w.input_scale).to(w.dtype)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.S), dtype=torch.float32, device=dev)
+
+    def step():
+        rm.ring_attn_fwd(q, k, v, w.P, w.causal, w.order, out=o, lse=lse, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize()
+    multi.barrier(dev)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev.index)
+    with sampler:
+        ms = time_on_stream(step, args.steps, stream)
+    torch.cuda.synchronize()
+    multi.barrier(dev)
+    if rm.native.rm_check_device_status(stream) != 0:
+        raise RuntimeError("device watchdog fired during the forward benchmark")
+    ms_max = multi.max_over_ranks(ms, dev)
+    bytes_in = sum(t.numel() * t.element_size() for t in (q, k, v))
+    bytes_out = o.numel() * o.element_size() + lse.numel() * 4
+    res = {"ms_total": ms_max, "launches": args.steps, "clocks": sampler.summary(),
+           "bytes_in": bytes_in, "bytes_out": bytes_out}
+
+    if not args.skip_e2e:
+        # end to end: pinned host inputs -> device, forward, result -> pinned host
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            rm.ring_attn_fwd(q, k, v, w.P, w.causal, w.order, out=o, lse=lse, stream=stream)
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        e2e_steps = max(3, min(args.steps, 50))
+        with torch.cuda.stream(stream):
+            e2e_step()
+            torch.cuda.synchronize()
+            multi.barrier(dev)
+            ms_e2e = time_on_stream(e2e_step, e2e_steps, stream)
+        multi.barrier(dev)
+        res["e2e"] = {"ms_per_step": multi.max_over_ranks(ms_e2e, dev) / e2e_steps,
+                      "steps": e2e_steps, "h2d": bytes_in, "d2h": bytes_out}
+    return res
+
+
+def bench_permute(args, dev, stream):
+    """Fused Q/K/V Ulysses permute (sequence- to head-sharded), 131072 tokens."""
+    import torch
+    import ring_ulysses_sequence_b200 as rm
+    from ring_ulysses_sequence_b200.synth import WORKLOADS
+    w = WORKLOADS["usp_fwd_bf16_S128k_u4r4"]
+    U, R = w.ulysses, w.P
+    q = torch.randn((w.B, w.S, w.H, w.D), device=dev).to(w.dtype)
+    k = torch.randn((w.B, w.S, w.Hkv, w.D), device=dev).to(w.dtype)
+    v = torch.randn((w.B, w.S, w.Hkv, w.D), device=dev).to(w.dtype)
+    outs = [torch.empty((w.B, w.H, w.S, w.D), device=dev, dtype=w.dtype),
+            torch.empty((w.B, w.Hkv, w.S, w.D), device=dev, dtype=w.dtype),
+            torch.empty((w.B, w.Hkv, w.S, w.D), device=dev, dtype=w.dtype)]
+
+    def step():
+        rm.ulysses_permute_qkv(q, k, v, U, R, "seq_to_head", outs=outs, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+    torch.cuda.synchronize()
+    steps = max(5, min(args.steps, 100))
+    ms = time_on_stream(step, steps, stream) / steps
+    moved = 2 * sum(t.numel() * t.element_size() for t in (q, k, v))  # read + write
+    return {"workload": w.name, "ms_per_launch": ms, "bytes_per_launch": moved,
+            "gbs": moved / ms / 1e6, "launches": steps + max(3, args.warmup)}
+
+
+def bench_backward(args, dev, stream):
+    """Ring attention backward on the 64k-token workload (B=2, 16 heads, P=16)."""
+    import torch
+    import ring_ulysses_sequence_b200 as rm
+    from ring_ulysses_sequence_b200.synth import WORKLOADS
+    w = WORKLOADS["ring_fwdbwd_bf16_S64k_causal_zigzag"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed)
+    q, k, v, do = ((torch.randn(s, generator=g, device=dev) * w.input_scale).to(w.dtype)
+                   for s in [(w.B, w.H, w.S, w.D), (w.B, w.Hkv, w.S, w.D),
+                             (w.B, w.Hkv, w.S, w.D), (w.B, w.H, w.S, w.D)])
+    o, lse = rm.ring_attn_fwd(q, k, v, w.P, w.causal, w.order, stream=stream)
+    ws = torch.empty(rm.native.rm_ring_attn_bwd_workspace_size(w.B, w.H, w.S), dtype=torch.uint8,
+                     device=dev)
+
+    def step():
+        return rm.ring_attn_bwd(q, k, v, o, lse, do, w.P, w.causal, w.order, workspace=ws,
+                                stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            step()
+    torch.cuda.synchronize()
+    steps = max(2, min(args.steps, 10))
+    ms = time_on_stream(step, steps, stream) / steps
+    return {"workload": w.name, "ms_per_step": ms, "tflops": w.bwd_flops() / ms / 1e9,
+            "flops_per_step": w.bwd_flops()}
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    from ring_ulysses_sequence_b200 import multi
+    from ring_ulysses_sequence_b200.synth import BENCH_WORKLOAD, WORKLOADS
+    rank, world, local = multi.env_ranks()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    multi.init("nccl", timeout_s=120, device=dev)
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.Stream(device=dev)
+    w = WORKLOADS[BENCH_WORKLOAD]
+    out = {}
+    try:
+        if args.only in ("all", "fwd"):
+            out["fwd"] = bench_forward(w, args, dev, stream)
+        if rank == 0 and args.only in ("all", "permute"):
+            out["permute"] = bench_permute(args, dev, stream)
+        if rank == 0 and args.only in ("all", "bwd"):
+            try:
+                out["bwd"] = bench_backward(args, dev, stream)
+            except Exception as e:  # backward not available: say so in the line
+                out["bwd"] = {"unavailable": str(e)[:200]}
+    finally:
+        multi.barrier(dev)
+    if rank != 0:
+        multi.shutdown()
+        return
+
+    line = {"metric": METRIC, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded N(0,1) x 0.5, bf16)",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup}
+    cfg = workload_config(w)
+    if "fwd" in out:
+        f = out["fwd"]
+        ms_step = f["ms_total"] / args.steps
+        flops = w.fwd_flops()
+        value = world * flops * args.steps / (f["ms_total"] * 1e-3) / 1e12
+        cfg["l2"] = (f"inputs {f['bytes_in'] / 1e6:.0f} MB + outputs {f['bytes_out'] / 1e6:.0f} MB "
+                     f"> {L2_BYTES >> 20} MiB L2 (no flush)")
+        sources = ["ring_ulysses_sequence_b200/csrc/fwd_tc.cu",
+                   "ring_ulysses_sequence_b200/csrc/common.cuh"]
+        peak = peaks["bf16_tflops"]
+        achieved = flops / (ms_step * 1e-3) / 1e12
+        line.update({
+            "value": value, "unit": "TFLOPS", "ms_per_step": ms_step,
+            "pct_of_peak": 100.0 * achieved / peak,
+            "roofline": {"bound": "tensor", "kernel": "ring_fwd_tc_kernel<128>",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak,
+                         "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)",
+                         "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peak),
+                         "frac_of_datasheet_2250": achieved / 2250.0,
+                         "flops_per_launch": flops,
+                         "traffic": profile_traffic("ring_fwd_tc_S32k_gqa_causal_zigzag.txt",
+                                                    sources)},
+            "clocks": f["clocks"],
+            "gpu_launches": f["launches"],
+        })
+        if "e2e" in f:
+            e = f["e2e"]
+            line["e2e"] = {"value": world * flops / (e["ms_per_step"] * 1e-3) / 1e12,
+                           "unit": "TFLOPS", "h2d_bytes_per_step": e["h2d"],
+                           "d2h_bytes_per_step": e["d2h"], "ms_per_step": e["ms_per_step"],
+                           "steps": e["steps"],
+                           "path": "pinned host q,k,v -> H2D -> rm_ring_attn_fwd -> D2H O, LSE"}
+    line["config"] = cfg
+    extra = {}
+    if "permute" in out:
+        p = out["permute"]
+        extra["ulysses_permute_qkv"] = {
+            "workload": p["workload"], "ms": p["ms_per_launch"], "GB/s": p["gbs"],
+            "roofline": {"bound": "hbm", "achieved": p["gbs"], "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": p["gbs"] / peaks["hbm_gbs"],
+                         "peak_source": f"{peak_src} hbm_gbs",
+                         "bytes_per_launch": p["bytes_per_launch"]}}
+    if "bwd" in out:
+        b = out["bwd"]
+        if "unavailable" in b:
+            extra["ring_attn_bwd"] = b
+        else:
+            extra["ring_attn_bwd"] = {
+                "workload": b["workload"], "ms": b["ms_per_step"], "TFLOPS": b["tflops"],
+                "roofline": {"bound": "tensor", "achieved": b["tflops"],
+                             "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                             "frac": b["tflops"] / peaks["bf16_tflops_sustained"],
+                             "peak_source": f"{peak_src} bf16_tflops_sustained"}}
+    if extra:
+        line["extra"] = extra
+    if world == 1 and not args.skip_cpu and args.only in ("all", "fwd"):
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+    multi.shutdown()
+
+
+if __name__ == "__main__":
+    main()
