@@ -109,11 +109,12 @@ RM_API rm_status rm_ring_attn_fwd(const void* q, const void* k, const void* v, v
  *
  *   q, k, v, o, dout : as in the forward (dtype; o is the forward's output)
  *   lse              : [B, H, S] float32 from the forward
- *   dq [B,H,S,D], dk, dv [B,Hkv,S,D] : float32, overwritten (zeroed first by
- *                      the library)
+ *   dq [B,H,S,D], dk, dv [B,Hkv,S,D] : float32, every element overwritten
+ *                      (no atomics: each is written exactly once)
  *   workspace        : device scratch of at least
  *                      rm_ring_attn_bwd_workspace_size(B, H, S) bytes, 256-byte
- *                      aligned, owned by the caller, contents need not be set.
+ *                      aligned, owned by the caller, contents need not be set
+ *                      (it receives Delta = rowsum(dO * O), [B, H, S] fp32).
  * Supported: dtype BF16, D in {64, 128}, same shape rules as the forward.
  */
 RM_API size_t rm_ring_attn_bwd_workspace_size(int B, int H, int S);

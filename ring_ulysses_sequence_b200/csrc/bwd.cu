@@ -1,12 +1,682 @@
-// Ring attention backward (placeholder until the tensor-core kernels land).
+// Ring attention backward, bf16 in / fp32 accumulate, on the sm_100a tensor
+// cores (axolotl-ringmaster README: flash-style reverse-ring backward, fp32
+// gradient accumulation across ring steps).
+//
+// Gradients of L = sum(dO * O), with P_ij = exp(scale q_i.k_j - LSE_i) over the
+// visible keys and Delta_i = <dO_i, O_i>:
+//   dV_j = sum_i P_ij dO_i            dS_ij = P_ij (<dO_i, v_j> - Delta_i)
+//   dK_j = scale sum_i dS_ij q_i      dQ_i  = scale sum_j dS_ij k_j
+// A KV head's dK/dV sum over the G query heads that share it.
+//
+// Three kernels, no atomics (every output element is written exactly once):
+//   bwd_delta_kernel   Delta = rowsum(dO * O)                      (HBM-bound)
+//   ring_bwd_dkdv      one 128-key tile of one KV head per work item (KV-
+//                      stationary). The tile's block travels the ring backwards:
+//                      at step t it visits the queries of rank (r + t) mod P,
+//                      every head of the group. Per query tile:
+//                        S^T = K Q^T, dP^T = V dO^T       (TMEM, fp32)
+//                        P^T, dS^T -> bf16 back into TMEM (compute warps)
+//                        dV += P^T dO, dK += dS^T Q       (TMEM A operand)
+//   ring_bwd_dq        one 128-query tile per work item (Q-stationary), key
+//                      tiles in ring order (i - t) mod P:
+//                        S = Q K^T, dP = dO V^T; dS -> bf16 in TMEM;
+//                        dQ += dS K
+// Warp roles as in the forward: warps 0-7 compute (two warpgroups splitting the
+// 128 columns of S), warp 8 issues UMMA, warp 9 issues TMA. TMEM (512 cols):
+// S [0,128), dP [128,256), accumulators at 256 and 384.
+#include <algorithm>
+
+#include "common.cuh"
 #include "internal.h"
+#include "tmap.h"
 
 namespace rm {
 
-cudaError_t launch_bwd(const AttnShape&, const void*, const void*, const void*, const void*,
-                       const float*, const void*, float*, float*, float*, float*,
-                       const LaunchCtx&) {
-    return cudaErrorNotSupported;
+namespace {
+
+constexpr int kT = 128;          // tile edge (rows of Q and of K/V)
+constexpr int kThreads = 320;
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp = 9;
+constexpr int kStages = 2;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct BCfg {
+    static constexpr int kTile = kT * D * 2;        // one bf16 tile
+    static constexpr int kBoxes = D / 64;
+    static constexpr int kBox = kT * 128;           // 16 KB swizzle box
+    // dK/dV kernel: K, V resident; stages of Q + dO + LSE + Delta
+    static constexpr int kStageKV = 2 * kTile + 2 * kT * 4;
+    static constexpr int kKvBarOff = 2 * kTile + kStages * kStageKV;
+    // dQ kernel: Q, dO resident; stages of K + V
+    static constexpr int kStageQ = 2 * kTile;
+    static constexpr int kQBarOff = 2 * kTile + kStages * kStageQ;
+    static constexpr int kSmemKV = kKvBarOff + 256 + 1024;
+    static constexpr int kSmemQ = kQBarOff + 256 + 1024;
+};
+
+enum : int { kSkip = 0, kDiag = 1, kFull = 2 };
+__device__ __forceinline__ int tile_class(int causal, int qpos, int kpos) {
+    if (!causal) return kFull;
+    return kpos > qpos ? kSkip : (kpos == qpos ? kDiag : kFull);
+}
+
+// TMEM column of K-step k (16 elements) of a bf16 operand written by the two
+// compute warpgroups: warpgroup w packs its 64 columns into [64w, 64w+32).
+__device__ __forceinline__ uint32_t packed_col(int k) { return k < 4 ? 8 * k : 64 + 8 * (k - 4); }
+
+struct BwdArgs {
+    CUtensorMap tm_q, tm_k, tm_v, tm_do;
+    const float* lse;
+    const float* delta;
+    float* dq;
+    float* dk;
+    float* dv;
+    unsigned* status;
+    unsigned long long timeout_ns;
+    int B, H, Hkv, S, P, causal, G, n_items;
+    float scale, scale_log2;
+    RingLayout lay;
+};
+
+struct Bars {
+    uint64_t res_full, res_empty, drain, acc_full;
+    uint64_t st_full[kStages], st_empty[kStages];
+    uint64_t s_full, p_full;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+// -------------------------------------------------------------------- dK / dV
+
+struct KvItem {
+    int b, g, kslot, kpos, rank;
+};
+
+// Key tiles in natural position order, earliest first (causal: they are seen
+// by the most query tiles).
+__device__ __forceinline__ KvItem decode_kv_item(const BwdArgs& a, int w) {
+    KvItem it;
+    const int nhu = a.B * a.Hkv;
+    const int unit = w / nhu, hu = w - unit * nhu;
+    it.b = hu / a.Hkv;
+    it.g = hu - it.b * a.Hkv;
+    it.kpos = unit * kT;
+    it.kslot = a.lay.slot_of_pos(it.kpos);
+    it.rank = it.kslot / a.lay.L;
+    return it;
+}
+
+// Query tiles (head, slot, class) that see a key tile, in reverse-ring order:
+// step t visits rank (r + t) mod P; heads of the group innermost.
+struct QIter {
+    RingLayout lay;
+    int rank, causal, kpos, G, g, t, u, hh, ntile, cls, qslot;
+    __device__ __forceinline__ QIter(const BwdArgs& a, const KvItem& it)
+        : lay(a.lay), rank(it.rank), causal(a.causal), kpos(it.kpos), G(a.G), g(it.g), t(0),
+          u(0), hh(a.G), ntile(a.lay.L / kT), cls(kSkip), qslot(0) {}
+    __device__ __forceinline__ bool next(int& h, int& slot, int& c) {
+        for (;;) {
+            if (hh < G) {
+                h = g * G + hh++;
+                slot = qslot;
+                c = cls;
+                return true;
+            }
+            if (t >= lay.P) return false;
+            int i = rank + t;
+            if (i >= lay.P) i -= lay.P;
+            qslot = i * lay.L + u * kT;
+            if (++u == ntile) { u = 0; ++t; }
+            cls = tile_class(causal, lay.pos_of_slot(qslot), kpos);
+            if (cls != kSkip) hh = 0;
+        }
+    }
+};
+
+template <int D>
+__device__ __forceinline__ void issue_tile_product(uint32_t tmem_d, uint32_t a_smem, uint32_t b_smem) {
+    // D[128 x 128] = A[128 x D] * B[128 x D]^T, both K-major in 128-byte swizzle boxes.
+    constexpr uint32_t idesc = umma_idesc_bf16(kT, kT, 0, 0);
+#pragma unroll
+    for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = (k >> 2) * BCfg<D>::kBox + (k & 3) * 32;
+        umma_ss(tmem_d, umma_desc_sw128(a_smem + off, 16, 1024), umma_desc_sw128(b_smem + off, 16, 1024),
+                idesc, k > 0 ? 1u : 0u);
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_acc_product(uint32_t tmem_acc, uint32_t tmem_a, uint32_t b_smem,
+                                                  bool accumulate) {
+    // ACC[128 x D] += A[128 x 128] (bf16 in TMEM) * B[128 x D] (row-major tile, MN-major operand).
+    constexpr uint32_t idesc = umma_idesc_bf16(kT, D, 0, 1);
+#pragma unroll
+    for (int k = 0; k < kT / 16; ++k)
+        umma_ts(tmem_acc, tmem_a + packed_col(k), umma_desc_sw128(b_smem + k * 2048, BCfg<D>::kBox, 1024),
+                idesc, (accumulate || k > 0) ? 1u : 0u);
+}
+
+// Stores N fp32 accumulator columns of this thread's TMEM row, times `mul`.
+template <int N>
+__device__ __forceinline__ void store_cols(uint32_t taddr, float* dst, float mul) {
+#pragma unroll 1
+    for (int cc = 0; cc < N; cc += 32) {
+        uint32_t v[32];
+        tmem_ld32(taddr + cc, v);
+        float4* d4 = reinterpret_cast<float4*>(dst + cc);
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            d4[c] = make_float4(__uint_as_float(v[4 * c]) * mul, __uint_as_float(v[4 * c + 1]) * mul,
+                                __uint_as_float(v[4 * c + 2]) * mul, __uint_as_float(v[4 * c + 3]) * mul);
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid_constant__ BwdArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    Bars& bars = *reinterpret_cast<Bars*>(smem + BCfg<D>::kKvBarOff);
+    const uint32_t k_smem = smem_u32(smem);
+    const uint32_t v_smem = k_smem + BCfg<D>::kTile;
+    const uint32_t st_smem = k_smem + 2 * BCfg<D>::kTile;  // stage s: Q, dO, LSE, Delta
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        bars.abort_flag = 0;
+        mbar_init(smem_u32(&bars.res_full), 1);
+        mbar_init(smem_u32(&bars.res_empty), 1);
+        mbar_init(smem_u32(&bars.drain), 1);
+        mbar_init(smem_u32(&bars.acc_full), 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(smem_u32(&bars.st_full[s]), 1);
+            mbar_init(smem_u32(&bars.st_empty[s]), 1);
+        }
+        mbar_init(smem_u32(&bars.s_full), 1);
+        mbar_init(smem_u32(&bars.p_full), 256);
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&bars.tmem_base), 512);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars.tmem_base;
+    const Watchdog wd{a.status, &bars.abort_flag, a.timeout_ns};
+
+    if (warp == kLoadWarp) {
+        if (lane == 0) {
+            prefetch_tmap(&a.tm_q);
+            prefetch_tmap(&a.tm_k);
+            prefetch_tmap(&a.tm_v);
+            prefetch_tmap(&a.tm_do);
+            uint32_t items = 0, fills = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x, ++items) {
+                const KvItem it = decode_kv_item(a, w);
+                if (items > 0) ok = mbar_wait(smem_u32(&bars.res_empty), (items - 1) & 1, wd);
+                if (!ok) break;
+                const int krow = (it.b * a.Hkv + it.g) * a.S + it.kslot;
+                mbar_arrive_expect_tx(smem_u32(&bars.res_full), 2 * BCfg<D>::kTile);
+                for (int bx = 0; bx < BCfg<D>::kBoxes; ++bx) {
+                    tma_load_2d(k_smem + bx * BCfg<D>::kBox, &a.tm_k, bx * 64, krow, smem_u32(&bars.res_full));
+                    tma_load_2d(v_smem + bx * BCfg<D>::kBox, &a.tm_v, bx * 64, krow, smem_u32(&bars.res_full));
+                }
+                QIter qi(a, it);
+                int h, qslot, cls;
+                while (ok && qi.next(h, qslot, cls)) {
+                    const int st = fills % kStages;
+                    const uint32_t use = fills / kStages;
+                    if (use > 0) ok = mbar_wait(smem_u32(&bars.st_empty[st]), (use - 1) & 1, wd);
+                    if (!ok) break;
+                    const uint32_t base = st_smem + st * BCfg<D>::kStageKV;
+                    const int qrow = (it.b * a.H + h) * a.S + qslot;
+                    const uint32_t bar = smem_u32(&bars.st_full[st]);
+                    mbar_arrive_expect_tx(bar, BCfg<D>::kStageKV);
+                    for (int bx = 0; bx < BCfg<D>::kBoxes; ++bx) {
+                        tma_load_2d(base + bx * BCfg<D>::kBox, &a.tm_q, bx * 64, qrow, bar);
+                        tma_load_2d(base + BCfg<D>::kTile + bx * BCfg<D>::kBox, &a.tm_do, bx * 64, qrow, bar);
+                    }
+                    bulk_load(base + 2 * BCfg<D>::kTile, a.lse + qrow, kT * 4, bar);
+                    bulk_load(base + 2 * BCfg<D>::kTile + kT * 4, a.delta + qrow, kT * 4, bar);
+                    ++fills;
+                }
+            }
+            if (!ok) {
+                volatile int no_abort = 0;
+                const Watchdog w2{a.status, &no_abort, a.timeout_ns};
+                for (uint32_t i = fills > kStages ? fills - kStages : 0; i < fills; ++i)
+                    (void)mbar_wait(smem_u32(&bars.st_full[i % kStages]), (i / kStages) & 1, w2);
+                if (items > 0) (void)mbar_wait(smem_u32(&bars.res_full), (items - 1) & 1, w2);
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 384;
+            uint32_t items = 0, uses = 0, p_cnt = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x, ++items) {
+                const KvItem it = decode_kv_item(a, w);
+                int n = 0;
+                {
+                    QIter qi(a, it);
+                    int h, s, c;
+                    while (qi.next(h, s, c)) ++n;
+                }
+                ok = mbar_wait(smem_u32(&bars.res_full), items & 1, wd);
+                if (!ok) break;
+                tc_fence_after();
+                for (int j = 0; j < n && ok; ++j) {
+                    const int st = uses % kStages;
+                    ok = mbar_wait(smem_u32(&bars.st_full[st]), (uses / kStages) & 1, wd);
+                    if (!ok) break;
+                    ++uses;
+                    tc_fence_after();
+                    const uint32_t q_addr = st_smem + st * BCfg<D>::kStageKV;
+                    const uint32_t do_addr = q_addr + BCfg<D>::kTile;
+                    issue_tile_product<D>(tS, k_smem, q_addr);     // S^T = K Q^T
+                    issue_tile_product<D>(tdP, v_smem, do_addr);   // dP^T = V dO^T
+                    umma_commit(smem_u32(&bars.s_full));
+                    ok = mbar_wait(smem_u32(&bars.p_full), (p_cnt++) & 1, wd);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_acc_product<D>(tdV, tS, do_addr, j > 0);   // dV += P^T dO
+                    issue_acc_product<D>(tdK, tdP, q_addr, j > 0);   // dK += dS^T Q
+                    umma_commit(smem_u32(&bars.st_empty[st]));
+                }
+                if (!ok) break;
+                umma_commit(smem_u32(&bars.acc_full));
+                umma_commit(smem_u32(&bars.res_empty));
+            }
+            umma_commit(smem_u32(&bars.drain));
+            volatile int no_abort = 0;
+            const Watchdog w2{a.status, &no_abort, a.timeout_ns};
+            (void)mbar_wait(smem_u32(&bars.drain), 0, w2);
+        }
+    } else {
+        const int wg = warp >> 2;               // which 64 query columns
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;      // key row of the tile = TMEM lane
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        const uint32_t tS = tmem + lane_off + 64 * wg;
+        const uint32_t tdP = tmem + lane_off + 128 + 64 * wg;
+        constexpr int HC = D / 2;               // accumulator columns per warpgroup
+        const uint32_t tdV = tmem + lane_off + 256 + HC * wg;
+        const uint32_t tdK = tmem + lane_off + 384 + HC * wg;
+        const float sl2 = a.scale_log2;
+        uint32_t uses = 0, s_cnt = 0, items = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x, ++items) {
+            const KvItem it = decode_kv_item(a, w);
+            QIter qi(a, it);
+            int h, qslot, cls;
+            while (ok && qi.next(h, qslot, cls)) {
+                const int st = uses % kStages;
+                ++uses;
+                const float* lse_s = reinterpret_cast<const float*>(
+                    smem + 2 * BCfg<D>::kTile + st * BCfg<D>::kStageKV + 2 * BCfg<D>::kTile);
+                const float* del_s = lse_s + kT;
+                ok = mbar_wait(smem_u32(&bars.s_full), (s_cnt++) & 1, wd);
+                if (!ok) break;
+                tc_fence_after();
+                uint32_t sv[64], dpv[64];
+                tmem_ld64(tS, sv);
+                tmem_ld64(tdP, dpv);
+                uint32_t pk[32], dsk[32];
+#pragma unroll
+                for (int c = 0; c < 64; c += 2) {
+                    const int q0 = 64 * wg + c;
+                    float p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lse_s[q0] * kLog2e));
+                    float p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -lse_s[q0 + 1] * kLog2e));
+                    if (cls == kDiag) {
+                        if (r > q0) p0 = 0.f;
+                        if (r > q0 + 1) p1 = 0.f;
+                    }
+                    const float d0 = p0 * (__uint_as_float(dpv[c]) - del_s[q0]);
+                    const float d1 = p1 * (__uint_as_float(dpv[c + 1]) - del_s[q0 + 1]);
+                    pk[c >> 1] = pack_bf16x2(p0, p1);
+                    dsk[c >> 1] = pack_bf16x2(d0, d1);
+                }
+                tmem_st32(tS, pk);
+                tmem_st32(tdP, dsk);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(smem_u32(&bars.p_full));
+            }
+            if (!ok) break;
+            ok = mbar_wait(smem_u32(&bars.acc_full), items & 1, wd);
+            if (!ok) break;
+            tc_fence_after();
+            const int64_t krow = (static_cast<int64_t>(it.b) * a.Hkv + it.g) * a.S + it.kslot + r;
+            store_cols<HC>(tdV, a.dv + krow * D + HC * wg, 1.0f);
+            store_cols<HC>(tdK, a.dk + krow * D + HC * wg, a.scale);
+        }
+    }
+
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// -------------------------------------------------------------------- dQ
+
+struct QItem {
+    int b, h, g, slot, pos, rank;
+};
+
+// Query tiles, latest natural position first when causal (the most key tiles).
+__device__ __forceinline__ QItem decode_q_item(const BwdArgs& a, int w) {
+    QItem it;
+    const int nhu = a.B * a.H;
+    const int unit = w / nhu, hu = w - unit * nhu;
+    it.b = hu / a.H;
+    it.h = hu - it.b * a.H;
+    it.g = it.h / a.G;
+    const int nu = a.causal ? (a.S / kT) - 1 - unit : unit;
+    it.pos = nu * kT;
+    it.slot = a.lay.slot_of_pos(it.pos);
+    it.rank = it.slot / a.lay.L;
+    return it;
+}
+
+// Key tiles a query tile sees, in ring order: step t visits owner (i - t) mod P.
+struct KIter {
+    RingLayout lay;
+    int rank, causal, qpos, t, u, ntile;
+    __device__ __forceinline__ KIter(const BwdArgs& a, const QItem& it)
+        : lay(a.lay), rank(it.rank), causal(a.causal), qpos(it.pos), t(0), u(0), ntile(a.lay.L / kT) {}
+    __device__ __forceinline__ bool next(int& kslot, int& cls) {
+        while (t < lay.P) {
+            const int ks = lay.owner(rank, t) * lay.L + u * kT;
+            if (++u == ntile) { u = 0; ++t; }
+            cls = tile_class(causal, qpos, lay.pos_of_slot(ks));
+            if (cls != kSkip) { kslot = ks; return true; }
+        }
+        return false;
+    }
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_constant__ BwdArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    Bars& bars = *reinterpret_cast<Bars*>(smem + BCfg<D>::kQBarOff);
+    const uint32_t q_smem = smem_u32(smem);
+    const uint32_t do_smem = q_smem + BCfg<D>::kTile;
+    const uint32_t st_smem = q_smem + 2 * BCfg<D>::kTile;  // stage s: K, V
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        bars.abort_flag = 0;
+        mbar_init(smem_u32(&bars.res_full), 1);
+        mbar_init(smem_u32(&bars.res_empty), 1);
+        mbar_init(smem_u32(&bars.drain), 1);
+        mbar_init(smem_u32(&bars.acc_full), 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(smem_u32(&bars.st_full[s]), 1);
+            mbar_init(smem_u32(&bars.st_empty[s]), 1);
+        }
+        mbar_init(smem_u32(&bars.s_full), 1);
+        mbar_init(smem_u32(&bars.p_full), 256);
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&bars.tmem_base), 512);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars.tmem_base;
+    const Watchdog wd{a.status, &bars.abort_flag, a.timeout_ns};
+
+    if (warp == kLoadWarp) {
+        if (lane == 0) {
+            prefetch_tmap(&a.tm_q);
+            prefetch_tmap(&a.tm_k);
+            prefetch_tmap(&a.tm_v);
+            prefetch_tmap(&a.tm_do);
+            uint32_t items = 0, fills = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x, ++items) {
+                const QItem it = decode_q_item(a, w);
+                if (items > 0) ok = mbar_wait(smem_u32(&bars.res_empty), (items - 1) & 1, wd);
+                if (!ok) break;
+                const int qrow = (it.b * a.H + it.h) * a.S + it.slot;
+                mbar_arrive_expect_tx(smem_u32(&bars.res_full), 2 * BCfg<D>::kTile);
+                for (int bx = 0; bx < BCfg<D>::kBoxes; ++bx) {
+                    tma_load_2d(q_smem + bx * BCfg<D>::kBox, &a.tm_q, bx * 64, qrow, smem_u32(&bars.res_full));
+                    tma_load_2d(do_smem + bx * BCfg<D>::kBox, &a.tm_do, bx * 64, qrow, smem_u32(&bars.res_full));
+                }
+                KIter ki(a, it);
+                int kslot, cls;
+                while (ok && ki.next(kslot, cls)) {
+                    const int st = fills % kStages;
+                    const uint32_t use = fills / kStages;
+                    if (use > 0) ok = mbar_wait(smem_u32(&bars.st_empty[st]), (use - 1) & 1, wd);
+                    if (!ok) break;
+                    const uint32_t base = st_smem + st * BCfg<D>::kStageQ;
+                    const int krow = (it.b * a.Hkv + it.g) * a.S + kslot;
+                    const uint32_t bar = smem_u32(&bars.st_full[st]);
+                    mbar_arrive_expect_tx(bar, BCfg<D>::kStageQ);
+                    for (int bx = 0; bx < BCfg<D>::kBoxes; ++bx) {
+                        tma_load_2d(base + bx * BCfg<D>::kBox, &a.tm_k, bx * 64, krow, bar);
+                        tma_load_2d(base + BCfg<D>::kTile + bx * BCfg<D>::kBox, &a.tm_v, bx * 64, krow, bar);
+                    }
+                    ++fills;
+                }
+            }
+            if (!ok) {
+                volatile int no_abort = 0;
+                const Watchdog w2{a.status, &no_abort, a.timeout_ns};
+                for (uint32_t i = fills > kStages ? fills - kStages : 0; i < fills; ++i)
+                    (void)mbar_wait(smem_u32(&bars.st_full[i % kStages]), (i / kStages) & 1, w2);
+                if (items > 0) (void)mbar_wait(smem_u32(&bars.res_full), (items - 1) & 1, w2);
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
+            uint32_t items = 0, uses = 0, p_cnt = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x, ++items) {
+                const QItem it = decode_q_item(a, w);
+                int n = 0;
+                {
+                    KIter ki(a, it);
+                    int ks, c;
+                    while (ki.next(ks, c)) ++n;
+                }
+                ok = mbar_wait(smem_u32(&bars.res_full), items & 1, wd);
+                if (!ok) break;
+                tc_fence_after();
+                for (int j = 0; j < n && ok; ++j) {
+                    const int st = uses % kStages;
+                    ok = mbar_wait(smem_u32(&bars.st_full[st]), (uses / kStages) & 1, wd);
+                    if (!ok) break;
+                    ++uses;
+                    tc_fence_after();
+                    const uint32_t k_addr = st_smem + st * BCfg<D>::kStageQ;
+                    const uint32_t v_addr = k_addr + BCfg<D>::kTile;
+                    issue_tile_product<D>(tS, q_smem, k_addr);     // S = Q K^T
+                    issue_tile_product<D>(tdP, do_smem, v_addr);   // dP = dO V^T
+                    umma_commit(smem_u32(&bars.s_full));
+                    ok = mbar_wait(smem_u32(&bars.p_full), (p_cnt++) & 1, wd);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_acc_product<D>(tdQ, tdP, k_addr, j > 0);   // dQ += dS K
+                    umma_commit(smem_u32(&bars.st_empty[st]));
+                }
+                if (!ok) break;
+                umma_commit(smem_u32(&bars.acc_full));
+                umma_commit(smem_u32(&bars.res_empty));
+            }
+            umma_commit(smem_u32(&bars.drain));
+            volatile int no_abort = 0;
+            const Watchdog w2{a.status, &no_abort, a.timeout_ns};
+            (void)mbar_wait(smem_u32(&bars.drain), 0, w2);
+        }
+    } else {
+        const int wg = warp >> 2;               // which 64 key columns
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;      // query row of the tile = TMEM lane
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        const uint32_t tS = tmem + lane_off + 64 * wg;
+        const uint32_t tdP = tmem + lane_off + 128 + 64 * wg;
+        constexpr int HC = D / 2;
+        const uint32_t tdQ = tmem + lane_off + 256 + HC * wg;
+        const float sl2 = a.scale_log2;
+        uint32_t s_cnt = 0, items = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x, ++items) {
+            const QItem it = decode_q_item(a, w);
+            const int64_t qrow = (static_cast<int64_t>(it.b) * a.H + it.h) * a.S + it.slot + r;
+            const float lse2 = a.lse[qrow] * kLog2e;
+            const float delta = a.delta[qrow];
+            KIter ki(a, it);
+            int kslot, cls;
+            while (ok && ki.next(kslot, cls)) {
+                ok = mbar_wait(smem_u32(&bars.s_full), (s_cnt++) & 1, wd);
+                if (!ok) break;
+                tc_fence_after();
+                uint32_t sv[64], dpv[64];
+                tmem_ld64(tS, sv);
+                tmem_ld64(tdP, dpv);
+                uint32_t dsk[32];
+#pragma unroll
+                for (int c = 0; c < 64; c += 2) {
+                    const int k0 = 64 * wg + c;
+                    float p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lse2));
+                    float p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -lse2));
+                    if (cls == kDiag) {
+                        if (k0 > r) p0 = 0.f;
+                        if (k0 + 1 > r) p1 = 0.f;
+                    }
+                    dsk[c >> 1] = pack_bf16x2(p0 * (__uint_as_float(dpv[c]) - delta),
+                                              p1 * (__uint_as_float(dpv[c + 1]) - delta));
+                }
+                tmem_st32(tdP, dsk);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(smem_u32(&bars.p_full));
+            }
+            if (!ok) break;
+            ok = mbar_wait(smem_u32(&bars.acc_full), items & 1, wd);
+            if (!ok) break;
+            tc_fence_after();
+            store_cols<HC>(tdQ, a.dq + qrow * D + HC * wg, a.scale);
+        }
+    }
+
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// -------------------------------------------------------------------- Delta
+
+// Delta_i = <dO_i, O_i> in fp32 from the bf16 rows; one warp per row.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_delta_kernel(const __nv_bfloat16* __restrict__ o,
+                                                        const __nv_bfloat16* __restrict__ dout,
+                                                        float* __restrict__ delta, int64_t rows) {
+    constexpr int PER = D / 32;  // elements per lane
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * 256) >> 5;
+    for (int64_t r = warp; r < rows; r += nwarps) {
+        const __nv_bfloat16* po = o + r * D + lane * PER;
+        const __nv_bfloat16* pd = dout + r * D + lane * PER;
+        float acc = 0.f;
+        if constexpr (PER == 4) {
+            const uint2 vo = *reinterpret_cast<const uint2*>(po);
+            const uint2 vd = *reinterpret_cast<const uint2*>(pd);
+            const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&vo);
+            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&vd);
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const float2 x = __bfloat1622float2(a2[i]), y = __bfloat1622float2(b2[i]);
+                acc = fmaf(x.x, y.x, fmaf(x.y, y.y, acc));
+            }
+        } else {
+            const __nv_bfloat162 x2 = *reinterpret_cast<const __nv_bfloat162*>(po);
+            const __nv_bfloat162 y2 = *reinterpret_cast<const __nv_bfloat162*>(pd);
+            const float2 x = __bfloat1622float2(x2), y = __bfloat1622float2(y2);
+            acc = fmaf(x.x, y.x, x.y * y.y);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) delta[r] = acc;
+    }
+}
+
+template <int D>
+cudaError_t launch_bwd_d(const AttnShape& sh, const BwdArgs& base, const void* o, const void* dout,
+                         float* delta, const LaunchCtx& ctx) {
+    cudaError_t e;
+    const int64_t rows = static_cast<int64_t>(sh.B) * sh.H * sh.S;
+    const int64_t dblocks = std::min<int64_t>((rows + 7) / 8, static_cast<int64_t>(ctx.num_sms) * 16);
+    bwd_delta_kernel<D><<<static_cast<unsigned>(dblocks), 256, 0, ctx.stream>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), delta, rows);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    BwdArgs a = base;
+    a.n_items = sh.B * sh.Hkv * (sh.S / kT);
+    if ((e = cudaFuncSetAttribute(ring_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  BCfg<D>::kSmemKV)) != cudaSuccess)
+        return e;
+    ring_bwd_dkdv_kernel<D><<<std::min(a.n_items, ctx.num_sms), kThreads, BCfg<D>::kSmemKV, ctx.stream>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    a.n_items = sh.B * sh.H * (sh.S / kT);
+    if ((e = cudaFuncSetAttribute(ring_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  BCfg<D>::kSmemQ)) != cudaSuccess)
+        return e;
+    ring_bwd_dq_kernel<D><<<std::min(a.n_items, ctx.num_sms), kThreads, BCfg<D>::kSmemQ, ctx.stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd(const AttnShape& sh, const void* q, const void* k, const void* v,
+                       const void* o, const float* lse, const void* dout, float* dq, float* dk,
+                       float* dv, float* delta, const LaunchCtx& ctx) {
+    BwdArgs a{};
+    cudaError_t e;
+    const uint64_t qrows = static_cast<uint64_t>(sh.B) * sh.H * sh.S;
+    const uint64_t kvrows = static_cast<uint64_t>(sh.B) * sh.Hkv * sh.S;
+    if ((e = make_tmap_bf16_rows(&a.tm_q, q, qrows, sh.D, kT, 64)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16_rows(&a.tm_do, dout, qrows, sh.D, kT, 64)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16_rows(&a.tm_k, k, kvrows, sh.D, kT, 64)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16_rows(&a.tm_v, v, kvrows, sh.D, kT, 64)) != cudaSuccess) return e;
+    a.lse = lse;
+    a.delta = delta;
+    a.dq = dq;
+    a.dk = dk;
+    a.dv = dv;
+    a.status = ctx.status_word;
+    a.timeout_ns = ctx.watchdog_ns;
+    a.B = sh.B;
+    a.H = sh.H;
+    a.Hkv = sh.Hkv;
+    a.S = sh.S;
+    a.P = sh.P;
+    a.causal = sh.causal;
+    a.G = sh.H / sh.Hkv;
+    a.scale = sh.scale;
+    a.scale_log2 = sh.scale * kLog2e;
+    a.lay = RingLayout{sh.S, sh.P, sh.S / sh.P, sh.zigzag ? sh.S / (2 * sh.P) : sh.S / sh.P, sh.zigzag};
+    return sh.D == 64 ? launch_bwd_d<64>(sh, a, o, dout, delta, ctx)
+                      : launch_bwd_d<128>(sh, a, o, dout, delta, ctx);
 }
 
 }  // namespace rm

@@ -1,0 +1,92 @@
+"""Ring attention backward on the GPU against the fp64 oracle's analytic gradients.
+
+The GPU gets O and LSE from its own forward (as a training step would); the
+oracle differentiates exact attention. Tolerances as for O: max-abs 2e-2,
+mean-abs 2e-3 on dQ, dK, dV (fp32 outputs of bf16 inputs).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import BF16_MAX_ABS, BF16_MEAN_ABS, assert_close, to_natural, to_rank_major
+from ring_ulysses_sequence_b200.synth import WORKLOADS, make_inputs, make_tensor, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_grads(qn, kn, vn, don, P, order, causal):
+    """Natural-order CPU inputs -> GPU forward + backward -> natural-order fp32 grads."""
+    import ring_ulysses_sequence_b200 as rm
+    q, k, v, do = (to_rank_major(t, P, order).cuda() for t in (qn, kn, vn, don))
+    o, lse = rm.ring_attn_fwd(q, k, v, P, causal, order)
+    dq, dk, dv = rm.ring_attn_bwd(q, k, v, o, lse, do, P, causal, order)
+    torch.cuda.synchronize()
+    assert rm.native.rm_check_device_status() == 0
+    return tuple(to_natural(t.cpu(), P, order) for t in (dq, dk, dv))
+
+
+def _inputs(B, H, Hkv, S, D, seed, scale=0.5):
+    q = make_tensor((B, H, S, D), seed, torch.bfloat16, scale)
+    k = make_tensor((B, Hkv, S, D), seed + 1, torch.bfloat16, scale)
+    v = make_tensor((B, Hkv, S, D), seed + 2, torch.bfloat16, scale)
+    do = make_tensor((B, H, S, D), seed + 3, torch.bfloat16, scale)
+    return q, k, v, do
+
+
+@pytest.mark.parametrize("B,H,Hkv,S,D,P,order,causal", [
+    (1, 2, 2, 1024, 128, 4, "zigzag", True),
+    (1, 4, 2, 1024, 128, 2, "zigzag", True),      # GQA: dK/dV summed over 2 heads
+    (2, 3, 1, 512, 64, 2, "contiguous", True),    # group 3, D = 64, B = 2
+    (1, 2, 2, 1024, 128, 4, "zigzag", False),
+    (1, 4, 1, 512, 128, 1, "zigzag", True),       # P = 1, MQA
+])
+def test_bwd_shapes_full(B, H, Hkv, S, D, P, order, causal):
+    q, k, v, do = _inputs(B, H, Hkv, S, D, 300 + S + H)
+    dq, dk, dv = gpu_grads(q, k, v, do, P, order, causal)
+    rdq, rdkv = oracle.attn_bwd(q.float(), k.float(), v.float(), do.float(), causal)
+    for b in range(B):
+        for h in range(H):
+            assert_close(dq[b, h].numpy(), rdq[(b, h)], BF16_MAX_ABS, BF16_MEAN_ABS, f"dQ[{b},{h}]")
+        for g in range(Hkv):
+            assert_close(dk[b, g].numpy(), rdkv[(b, g)][0], BF16_MAX_ABS, BF16_MEAN_ABS, f"dK[{b},{g}]")
+            assert_close(dv[b, g].numpy(), rdkv[(b, g)][1], BF16_MAX_ABS, BF16_MEAN_ABS, f"dV[{b},{g}]")
+    # identities of the exact gradient, up to the bf16 tolerance:
+    # sum_j dK_j = 0, sum_j dV_j = sum over the group's heads of sum_i dO_i
+    G = H // Hkv
+    dsum = do.float().reshape(B, Hkv, G, S, D).sum(dim=(2, 3))
+    assert_close(dv.sum(dim=2).numpy(), dsum.numpy(), 0.5)
+    assert float(dk.sum(dim=2).abs().max()) < 0.5
+
+
+def test_bwd_deterministic():
+    import ring_ulysses_sequence_b200 as rm
+    q, k, v, do = (to_rank_major(t, 4, "zigzag").cuda() for t in _inputs(1, 4, 2, 1024, 128, 77))
+    o, lse = rm.ring_attn_fwd(q, k, v, 4, True, "zigzag")
+    a = rm.ring_attn_bwd(q, k, v, o, lse, do, 4, True, "zigzag")
+    b = rm.ring_attn_bwd(q, k, v, o, lse, do, 4, True, "zigzag")
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_bwd_workload_sampled():
+    """B=2, H=Hkv=16, S=65536, D=128, P=16 zigzag, causal: dQ on seeded query rows
+    of every head; dK/dV on seeded key rows of two seeded KV heads."""
+    w = WORKLOADS["ring_fwdbwd_bf16_S64k_causal_zigzag"]
+    q, k, v, do = make_inputs(w)
+    dq, dk, dv = gpu_grads(q, k, v, do, w.P, w.order, w.causal)
+    qrows = sample_rows(w.S, 64, w.seed + 1000, w.chunk)
+    krows = sample_rows(w.S, 64, w.seed + 2000, w.chunk)
+    rng = np.random.default_rng(w.seed + 3000)
+    kv_heads = [(int(rng.integers(w.B)), int(rng.integers(w.Hkv))) for _ in range(2)]
+    q_heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+    rdq, rdkv = oracle.attn_bwd(q.float(), k.float(), v.float(), do.float(), True, qrows=qrows,
+                                krows=krows, heads=(q_heads, kv_heads))
+    for (b, h) in q_heads:
+        assert_close(dq[b, h][qrows].numpy(), rdq[(b, h)], BF16_MAX_ABS, BF16_MEAN_ABS, f"dQ[{b},{h}]")
+    for (b, g) in kv_heads:
+        assert_close(dk[b, g][krows].numpy(), rdkv[(b, g)][0], BF16_MAX_ABS, BF16_MEAN_ABS, f"dK[{b},{g}]")
+        assert_close(dv[b, g][krows].numpy(), rdkv[(b, g)][1], BF16_MAX_ABS, BF16_MEAN_ABS, f"dV[{b},{g}]")
+    # properties at full size: sum_j dK_j = 0 and sum_j dV_j = sum_i dO_i per head
+    assert float(dk.sum(dim=2).abs().max()) < 1.0
+    assert_close(dv.sum(dim=2).numpy(), do.float().sum(dim=2).numpy(), 1.0)
