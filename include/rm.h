@@ -126,6 +126,38 @@ RM_API rm_status rm_ring_attn_bwd(const void* q, const void* k, const void* v, c
                            rm_dtype dtype, float scale, cudaStream_t stream);
 
 /*
+ * rm_ring_attn_bwd_noalloc — rm_ring_attn_bwd for callers that cannot allocate.
+ *
+ * The pages have no counterpart of this call; it serves library users. Some
+ * callers of this code cannot call cudaMalloc: a plugin inside a host
+ * framework that reserved all device memory up front and hands out only the
+ * tensors themselves, or a latency-critical loop where an allocation (which
+ * may synchronise the device or fail) is not allowed. This entry point takes
+ * the same tensors as rm_ring_attn_bwd but no workspace: its scratch (the
+ * Delta rows) lives in a static device array of the library that holds
+ * 2,097,152 fp32 values (8 MiB). Every GPU that loads the library keeps that
+ * array until the process exits.
+ *
+ *   Arguments, layouts, outputs and status codes as rm_ring_attn_bwd.
+ *   Limit: B * H * S <= 2,097,152; larger problems return RM_ERR_UNSUPPORTED
+ *   before anything is launched.
+ *   The first call on a device looks up the array's device address (a CUDA
+ *   runtime query, no allocation); make that first call before any stream
+ *   capture begins on that device.
+ *   All calls on a device share the one array, which keeps the last call's
+ *   contents. The backward rewrites the whole scratch it reads, so nothing
+ *   has to be cleared, but calls that overlap on the GPU (for example on two
+ *   streams) race on it and give undefined results: serialise them.
+ *   Nothing is allocated: no cudaMalloc, no cudaFree, no allocating library
+ *   routine.
+ */
+RM_API rm_status rm_ring_attn_bwd_noalloc(const void* q, const void* k, const void* v,
+                                          const void* o, const float* lse, const void* dout,
+                                          float* dq, float* dk, float* dv, int B, int H, int Hkv,
+                                          int S, int D, int P, int causal, rm_order order,
+                                          rm_dtype dtype, float scale, cudaStream_t stream);
+
+/*
  * rm_lse_merge — fold one partial (O, LSE) into a running pair, row by row,
  * in place ("DeDLOC Guide", section 3 alpha/beta rescaling, in the
  * normalised-output form of Step 3's merge):

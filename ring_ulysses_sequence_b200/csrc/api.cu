@@ -51,6 +51,34 @@ static rm_status get_ctx(cudaStream_t stream, LaunchCtx* ctx) {
     return RM_OK;
 }
 
+// Scratch of rm_ring_attn_bwd_noalloc: the Delta rows (B * H * S fp32 values)
+// of the backward, at most kNoAllocMaxRows of them (8 MiB). It is a static
+// device array, so every GPU that loads this library holds it until the
+// process exits; all calls on a device share it.
+constexpr size_t kNoAllocMaxRows = static_cast<size_t>(1) << 21;
+static __device__ __align__(256) float g_noalloc_delta[kNoAllocMaxRows];
+
+// Device address of g_noalloc_delta on the current device. In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device, with that device current, and cached.
+static rm_status noalloc_scratch(float** out) {
+    static std::mutex mu;
+    static float* addr[128] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= 128) return RM_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_delta);
+        if (e != cudaSuccess) return cuda_fail(e);
+        addr[dev] = static_cast<float*>(p);
+    }
+    *out = addr[dev];
+    return RM_OK;
+}
+
 static bool valid_order(rm_order o) { return o == RM_ORDER_CONTIGUOUS || o == RM_ORDER_ZIGZAG; }
 
 // Shared shape rules of the forward and backward.
@@ -169,6 +197,29 @@ rm_status rm_ring_attn_bwd(const void* q, const void* k, const void* v, const vo
     AttnShape sh{B, H, Hkv, S, D, P, causal ? 1 : 0, order == RM_ORDER_ZIGZAG ? 1 : 0, scale};
     cudaError_t e = launch_bwd(sh, q, k, v, o, lse, dout, dq, dk, dv,
                                static_cast<float*>(workspace), ctx);
+    return e == cudaSuccess ? RM_OK : cuda_fail(e);
+}
+
+rm_status rm_ring_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                   const float* lse, const void* dout, float* dq, float* dk,
+                                   float* dv, int B, int H, int Hkv, int S, int D, int P, int causal,
+                                   rm_order order, rm_dtype dtype, float scale, cudaStream_t stream) {
+    rm_status st = check_attn(q, k, v, B, H, Hkv, S, D, P, order, dtype, scale, 128);
+    if (st != RM_OK) return st;
+    if (dtype != RM_DTYPE_BF16) return RM_ERR_UNSUPPORTED;
+    if (B == 0 || S == 0) return RM_OK;
+    const void* ptrs[] = {o, lse, dout, dq, dk, dv};
+    for (const void* p : ptrs)
+        if (!p || !aligned16(p)) return RM_ERR_INVALID_ARG;
+    if (static_cast<size_t>(B) * H * S > kNoAllocMaxRows) return RM_ERR_UNSUPPORTED;
+    LaunchCtx ctx;
+    if ((st = get_ctx(stream, &ctx)) != RM_OK) return st;
+    float* scratch = nullptr;
+    if ((st = noalloc_scratch(&scratch)) != RM_OK) return st;
+    AttnShape sh{B, H, Hkv, S, D, P, causal ? 1 : 0, order == RM_ORDER_ZIGZAG ? 1 : 0, scale};
+    // Delta is rewritten in full by the backward's first kernel, so the
+    // previous call's contents need no clearing.
+    cudaError_t e = launch_bwd(sh, q, k, v, o, lse, dout, dq, dk, dv, scratch, ctx);
     return e == cudaSuccess ? RM_OK : cuda_fail(e);
 }
 

@@ -24,6 +24,8 @@ SIGNATURES = {
     "rm_ring_attn_bwd_workspace_size": (_sz, [_i, _i, _i]),
     "rm_ring_attn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                               _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
+    "rm_ring_attn_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                      _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "rm_lse_merge": (_i, [_vp, _vp, _vp, _vp, _i64, _i, _vp]),
     "rm_ulysses_permute": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "rm_ulysses_permute_qkv": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
@@ -105,6 +107,13 @@ def rm_ring_attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_byt
     return _call("rm_ring_attn_bwd", _p(q), _p(k), _p(v), _p(o), _p(lse), _p(dout), _p(dq),
                  _p(dk), _p(dv), _p(workspace), workspace_bytes, B, H, Hkv, S, D, P, int(causal),
                  order, dtype, scale, _s(stream))
+
+
+def rm_ring_attn_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, H, Hkv, S, D, P, causal,
+                             order, dtype, scale, stream=None):
+    return _call("rm_ring_attn_bwd_noalloc", _p(q), _p(k), _p(v), _p(o), _p(lse), _p(dout),
+                 _p(dq), _p(dk), _p(dv), B, H, Hkv, S, D, P, int(causal), order, dtype, scale,
+                 _s(stream))
 
 
 def rm_lse_merge(o_acc, lse_acc, o_part, lse_part, rows, D, stream=None):
