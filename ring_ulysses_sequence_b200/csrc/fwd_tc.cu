@@ -112,22 +112,41 @@ __device__ __forceinline__ int tile_class(int causal, int qpos, int kpos) {
 }
 
 // Key tiles of an item in ring order: step t visits owner (rank - t) mod P.
+// An owner's block is one run (contiguous order) or two runs (zigzag: chunk r
+// then chunk 2P-1-r) of consecutive natural positions, so the tiles a causal
+// query tile can see form a prefix of each run: O(1) work per tile returned,
+// no division.
 struct KvIter {
-    RingLayout lay;
-    int rank, causal, pos0, pos1, t, u, ntile;
-    __device__ __forceinline__ KvIter(const TcArgs& a, const Item& it)
-        : lay(a.lay), rank(it.rank), causal(a.causal), pos0(it.pos0), pos1(it.pos1), t(0), u(0),
-          ntile(a.lay.L / kBN) {}
+    const TcArgs* a;   // layout read from the kernel parameters, not copied
+    int rank, pos0, pos1, t, run, u, u_end, s0, p0;
+    __device__ __forceinline__ KvIter(const TcArgs& args, const Item& it)
+        : a(&args), rank(it.rank), pos0(it.pos0), pos1(it.pos1), t(0), run(-1), u(0), u_end(0),
+          s0(0), p0(0) {}
     __device__ __forceinline__ bool next(int& kslot, int& c0, int& c1) {
-        while (t < lay.P) {
-            const int ks = lay.owner(rank, t) * lay.L + u * kBN;
-            if (++u == ntile) { u = 0; ++t; }
-            const int kp = lay.pos_of_slot(ks);
-            c0 = tile_class(causal, pos0, kp);
-            c1 = tile_class(causal, pos1, kp);
-            if (c0 != kSkip || c1 != kSkip) { kslot = ks; return true; }
+        const RingLayout& lay = a->lay;
+        while (u >= u_end) {
+            const int runs = lay.zigzag ? 2 : 1;
+            if (++run == runs) {  // run starts at -1, so the first call opens run 0 of step 0
+                run = 0;
+                if (++t == lay.P) return false;
+            }
+            const int r = lay.owner(rank, t);
+            const int ctiles = (lay.zigzag ? lay.c : lay.L) / kBN;
+            s0 = r * lay.L + run * lay.c;
+            p0 = lay.zigzag ? (run == 0 ? r * lay.c : (2 * lay.P - 1 - r) * lay.c) : r * lay.L;
+            u = 0;
+            u_end = ctiles;
+            if (a->causal) {
+                const int vis = ((max(pos0, pos1) - p0) >> 7) + 1;  // tiles at or before the query
+                u_end = min(ctiles, max(vis, 0));
+            }
         }
-        return false;
+        const int kp = p0 + u * kBN;
+        kslot = s0 + u * kBN;
+        ++u;
+        c0 = tile_class(a->causal, pos0, kp);
+        c1 = tile_class(a->causal, pos1, kp);
+        return true;
     }
 };
 
@@ -254,12 +273,10 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
             bool ok = true;
             for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x) {
                 const Item it = decode_item(a, w);
-                int n = 0;
-                {
-                    KvIter kv(a, it);
-                    int ks, c0, c1;
-                    while (kv.next(ks, c0, c1)) ++n;
-                }
+                KvIter kv(a, it);
+                int ks, c0, c1;
+                bool have_cur = kv.next(ks, c0, c1);   // tile 0 (every item has one)
+                bool have_next = kv.next(ks, c0, c1);  // tile 1
                 ok = mbar_wait(smem_u32(&bars.q_full), q_iter & 1, wd);
                 if (!ok) break;
                 ++q_iter;
@@ -274,8 +291,9 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
                 issue_qk<D>(tS[1], q_smem + Cfg<D>::kTileBytes, kv_smem + stK * Cfg<D>::kTileBytes);
                 umma_commit(smem_u32(&bars.s_full[1]));
                 umma_commit(smem_u32(&bars.kv_empty[stK]));
-                if (n == 1) umma_commit(smem_u32(&bars.q_empty));
-                for (int j = 0; j < n && ok; ++j) {
+                if (!have_next) umma_commit(smem_u32(&bars.q_empty));
+                for (int j = 0; have_cur && ok; ++j) {
+                    const bool have_next2 = have_next && kv.next(ks, c0, c1);  // tile j + 2
                     const uint32_t stV = kv_iter % kStages;
                     ok = mbar_wait(smem_u32(&bars.kv_full[stV]), (kv_iter / kStages) & 1, wd);
                     if (!ok) break;
@@ -285,9 +303,8 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
                     if (!ok) break;
                     tc_fence_after();
                     issue_pv<D>(tO[0], tS[0], v_addr, j > 0);
-                    if (j == n - 1) umma_commit(smem_u32(&bars.o_full[0]));
-                    const bool more = j + 1 < n;
-                    if (more) {
+                    if (!have_next) umma_commit(smem_u32(&bars.o_full[0]));
+                    if (have_next) {
                         stK = kv_iter % kStages;
                         ok = mbar_wait(smem_u32(&bars.kv_full[stK]), (kv_iter / kStages) & 1, wd);
                         if (!ok) break;
@@ -301,14 +318,16 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
                     tc_fence_after();
                     issue_pv<D>(tO[1], tS[1], v_addr, j > 0);
                     umma_commit(smem_u32(&bars.kv_empty[stV]));
-                    if (j == n - 1) umma_commit(smem_u32(&bars.o_full[1]));
-                    if (more) {
+                    if (!have_next) umma_commit(smem_u32(&bars.o_full[1]));
+                    if (have_next) {
                         issue_qk<D>(tS[1], q_smem + Cfg<D>::kTileBytes,
                                     kv_smem + stK * Cfg<D>::kTileBytes);
                         umma_commit(smem_u32(&bars.s_full[1]));
                         umma_commit(smem_u32(&bars.kv_empty[stK]));
-                        if (j + 1 == n - 1) umma_commit(smem_u32(&bars.q_empty));
+                        if (!have_next2) umma_commit(smem_u32(&bars.q_empty));
                     }
+                    have_cur = have_next;
+                    have_next = have_next2;
                 }
             }
             // Every product issued must finish before TMEM is released.
