@@ -109,28 +109,43 @@ __device__ __forceinline__ KvItem decode_kv_item(const BwdArgs& a, int w) {
 }
 
 // Query tiles (head, slot, class) that see a key tile, in reverse-ring order:
-// step t visits rank (r + t) mod P; heads of the group innermost.
+// step t visits rank (r + t) mod P; heads of the group innermost. A rank's
+// block is one (contiguous) or two (zigzag) runs of consecutive positions, and
+// the query tiles that see a causal key tile form a suffix of each run: O(1)
+// work per returned tile, no division.
 struct QIter {
-    RingLayout lay;
-    int rank, causal, kpos, G, g, t, u, hh, ntile, cls, qslot;
-    __device__ __forceinline__ QIter(const BwdArgs& a, const KvItem& it)
-        : lay(a.lay), rank(it.rank), causal(a.causal), kpos(it.kpos), G(a.G), g(it.g), t(0),
-          u(0), hh(a.G), ntile(a.lay.L / kT), cls(kSkip), qslot(0) {}
+    const BwdArgs* a;
+    int rank, kpos, g, t, run, u, u_end, s0, p0, hh, cls, qslot;
+    __device__ __forceinline__ QIter(const BwdArgs& args, const KvItem& it)
+        : a(&args), rank(it.rank), kpos(it.kpos), g(it.g), t(0), run(-1), u(0), u_end(0), s0(0),
+          p0(0), hh(args.G), cls(kSkip), qslot(0) {}
     __device__ __forceinline__ bool next(int& h, int& slot, int& c) {
+        const RingLayout& lay = a->lay;
         for (;;) {
-            if (hh < G) {
-                h = g * G + hh++;
+            if (hh < a->G) {
+                h = g * a->G + hh++;
                 slot = qslot;
                 c = cls;
                 return true;
             }
-            if (t >= lay.P) return false;
-            int i = rank + t;
-            if (i >= lay.P) i -= lay.P;
-            qslot = i * lay.L + u * kT;
-            if (++u == ntile) { u = 0; ++t; }
-            cls = tile_class(causal, lay.pos_of_slot(qslot), kpos);
-            if (cls != kSkip) hh = 0;
+            while (u >= u_end) {
+                const int runs = lay.zigzag ? 2 : 1;
+                if (++run == runs) {  // run starts at -1: the first call opens run 0 of step 0
+                    run = 0;
+                    if (++t == lay.P) return false;
+                }
+                int i = rank + t;
+                if (i >= lay.P) i -= lay.P;
+                const int ctiles = (lay.zigzag ? lay.c : lay.L) / kT;
+                s0 = i * lay.L + run * lay.c;
+                p0 = lay.zigzag ? (run == 0 ? i * lay.c : (2 * lay.P - 1 - i) * lay.c) : i * lay.L;
+                u_end = ctiles;
+                u = a->causal ? min(ctiles, max((kpos - p0) >> 7, 0)) : 0;  // first tile at or after the key
+            }
+            qslot = s0 + u * kT;
+            cls = tile_class(a->causal, p0 + u * kT, kpos);
+            ++u;
+            hh = 0;
         }
     }
 };
@@ -261,16 +276,12 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
             bool ok = true;
             for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x, ++items) {
                 const KvItem it = decode_kv_item(a, w);
-                int n = 0;
-                {
-                    QIter qi(a, it);
-                    int h, s, c;
-                    while (qi.next(h, s, c)) ++n;
-                }
+                QIter qi(a, it);
+                int qh, qs, qc;
                 ok = mbar_wait(smem_u32(&bars.res_full), items & 1, wd);
                 if (!ok) break;
                 tc_fence_after();
-                for (int j = 0; j < n && ok; ++j) {
+                for (int j = 0; ok && qi.next(qh, qs, qc); ++j) {
                     const int st = uses % kStages;
                     ok = mbar_wait(smem_u32(&bars.st_full[st]), (uses / kStages) & 1, wd);
                     if (!ok) break;
@@ -323,26 +334,31 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
                 ok = mbar_wait(smem_u32(&bars.s_full), (s_cnt++) & 1, wd);
                 if (!ok) break;
                 tc_fence_after();
-                uint32_t sv[64], dpv[64];
-                tmem_ld64(tS, sv);
-                tmem_ld64(tdP, dpv);
-                uint32_t pk[32], dsk[32];
+                // two quarters of 32 query columns: load S^T and dP^T, write
+                // bf16 P^T and dS^T over S^T/dP^T columns already read
 #pragma unroll
-                for (int c = 0; c < 64; c += 2) {
-                    const int q0 = 64 * wg + c;
-                    float p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lse_s[q0] * kLog2e));
-                    float p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -lse_s[q0 + 1] * kLog2e));
-                    if (cls == kDiag) {
-                        if (r > q0) p0 = 0.f;
-                        if (r > q0 + 1) p1 = 0.f;
+                for (int qq = 0; qq < 2; ++qq) {
+                    uint32_t sv[32], dpv[32];
+                    tmem_ld32(tS + 32 * qq, sv);
+                    tmem_ld32(tdP + 32 * qq, dpv);
+                    uint32_t pk[16], dsk[16];
+#pragma unroll
+                    for (int c = 0; c < 32; c += 2) {
+                        const int q0 = 64 * wg + 32 * qq + c;
+                        float p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lse_s[q0] * kLog2e));
+                        float p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -lse_s[q0 + 1] * kLog2e));
+                        if (cls == kDiag) {
+                            if (r > q0) p0 = 0.f;
+                            if (r > q0 + 1) p1 = 0.f;
+                        }
+                        const float d0 = p0 * (__uint_as_float(dpv[c]) - del_s[q0]);
+                        const float d1 = p1 * (__uint_as_float(dpv[c + 1]) - del_s[q0 + 1]);
+                        pk[c >> 1] = pack_bf16x2(p0, p1);
+                        dsk[c >> 1] = pack_bf16x2(d0, d1);
                     }
-                    const float d0 = p0 * (__uint_as_float(dpv[c]) - del_s[q0]);
-                    const float d1 = p1 * (__uint_as_float(dpv[c + 1]) - del_s[q0 + 1]);
-                    pk[c >> 1] = pack_bf16x2(p0, p1);
-                    dsk[c >> 1] = pack_bf16x2(d0, d1);
+                    tmem_st16(tS + 16 * qq, pk);
+                    tmem_st16(tdP + 16 * qq, dsk);
                 }
-                tmem_st32(tS, pk);
-                tmem_st32(tdP, dsk);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(smem_u32(&bars.p_full));
@@ -385,20 +401,32 @@ __device__ __forceinline__ QItem decode_q_item(const BwdArgs& a, int w) {
     return it;
 }
 
-// Key tiles a query tile sees, in ring order: step t visits owner (i - t) mod P.
+// Key tiles a query tile sees, in ring order: step t visits owner (i - t) mod P;
+// within each run of an owner's block the visible tiles are a prefix.
 struct KIter {
-    RingLayout lay;
-    int rank, causal, qpos, t, u, ntile;
-    __device__ __forceinline__ KIter(const BwdArgs& a, const QItem& it)
-        : lay(a.lay), rank(it.rank), causal(a.causal), qpos(it.pos), t(0), u(0), ntile(a.lay.L / kT) {}
+    const BwdArgs* a;
+    int rank, qpos, t, run, u, u_end, s0, p0;
+    __device__ __forceinline__ KIter(const BwdArgs& args, const QItem& it)
+        : a(&args), rank(it.rank), qpos(it.pos), t(0), run(-1), u(0), u_end(0), s0(0), p0(0) {}
     __device__ __forceinline__ bool next(int& kslot, int& cls) {
-        while (t < lay.P) {
-            const int ks = lay.owner(rank, t) * lay.L + u * kT;
-            if (++u == ntile) { u = 0; ++t; }
-            cls = tile_class(causal, qpos, lay.pos_of_slot(ks));
-            if (cls != kSkip) { kslot = ks; return true; }
+        const RingLayout& lay = a->lay;
+        while (u >= u_end) {
+            const int runs = lay.zigzag ? 2 : 1;
+            if (++run == runs) {
+                run = 0;
+                if (++t == lay.P) return false;
+            }
+            const int r = lay.owner(rank, t);
+            const int ctiles = (lay.zigzag ? lay.c : lay.L) / kT;
+            s0 = r * lay.L + run * lay.c;
+            p0 = lay.zigzag ? (run == 0 ? r * lay.c : (2 * lay.P - 1 - r) * lay.c) : r * lay.L;
+            u = 0;
+            u_end = a->causal ? min(ctiles, max(((qpos - p0) >> 7) + 1, 0)) : ctiles;
         }
-        return false;
+        kslot = s0 + u * kT;
+        cls = tile_class(a->causal, qpos, p0 + u * kT);
+        ++u;
+        return true;
     }
 };
 
@@ -488,16 +516,12 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
             bool ok = true;
             for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x, ++items) {
                 const QItem it = decode_q_item(a, w);
-                int n = 0;
-                {
-                    KIter ki(a, it);
-                    int ks, c;
-                    while (ki.next(ks, c)) ++n;
-                }
+                KIter ki(a, it);
+                int ks, kc;
                 ok = mbar_wait(smem_u32(&bars.res_full), items & 1, wd);
                 if (!ok) break;
                 tc_fence_after();
-                for (int j = 0; j < n && ok; ++j) {
+                for (int j = 0; ok && ki.next(ks, kc); ++j) {
                     const int st = uses % kStages;
                     ok = mbar_wait(smem_u32(&bars.st_full[st]), (uses / kStages) & 1, wd);
                     if (!ok) break;
