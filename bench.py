@@ -47,6 +47,8 @@ def parse_args():
                    help="restrict to one kernel (used for profiling runs)")
     p.add_argument("--skip-cpu", action="store_true", help="skip the CPU oracle baseline")
     p.add_argument("--skip-e2e", action="store_true")
+    p.add_argument("--bwd-heads", type=int, default=None,
+                   help="heads of the backward case (default: the workload's; smaller for profiling)")
     args = p.parse_args()
     if args.warmup < 3 and args.only == "all":
         p.error("at least 3 warm-up steps")
@@ -346,6 +348,10 @@ def bench_backward(args, dev, stream):
     import ring_ulysses_sequence_b200 as rm
     from ring_ulysses_sequence_b200.synth import WORKLOADS
     w = WORKLOADS["ring_fwdbwd_bf16_S64k_causal_zigzag"]
+    if args.bwd_heads:
+        import dataclasses
+        w = dataclasses.replace(w, B=1, H=args.bwd_heads, Hkv=args.bwd_heads,
+                                name=f"{w.name}_B1_H{args.bwd_heads}")
     g = torch.Generator(device=dev)
     g.manual_seed(w.seed)
     q, k, v, do = ((torch.randn(s, generator=g, device=dev) * w.input_scale).to(w.dtype)
