@@ -335,26 +335,42 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
                 if (!ok) break;
                 tc_fence_after();
                 // two quarters of 32 query columns: load S^T and dP^T, write
-                // bf16 P^T and dS^T over S^T/dP^T columns already read
+                // bf16 P^T and dS^T over S^T/dP^T columns already read. LSE and
+                // Delta of the columns come four at a time from shared memory;
+                // the arithmetic runs on packed fp32 pairs.
+                const uint64_t sl2x2 = pk2(sl2, sl2);
+                const uint64_t nlog2e = pk2(-kLog2e, -kLog2e);
 #pragma unroll
                 for (int qq = 0; qq < 2; ++qq) {
                     uint32_t sv[32], dpv[32];
                     tmem_ld32(tS + 32 * qq, sv);
                     tmem_ld32(tdP + 32 * qq, dpv);
+                    const float4* lse4 = reinterpret_cast<const float4*>(lse_s + 64 * wg + 32 * qq);
+                    const float4* del4 = reinterpret_cast<const float4*>(del_s + 64 * wg + 32 * qq);
                     uint32_t pk[16], dsk[16];
 #pragma unroll
-                    for (int c = 0; c < 32; c += 2) {
-                        const int q0 = 64 * wg + 32 * qq + c;
-                        float p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lse_s[q0] * kLog2e));
-                        float p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -lse_s[q0 + 1] * kLog2e));
-                        if (cls == kDiag) {
-                            if (r > q0) p0 = 0.f;
-                            if (r > q0 + 1) p1 = 0.f;
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        const float4 L = lse4[c4], Dl = del4[c4];
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const int c = 4 * c4 + 2 * hh;
+                            const uint64_t lse2 = mul2(hh ? pk2(L.z, L.w) : pk2(L.x, L.y), nlog2e);
+                            float x0, x1;
+                            upk2(fma2(pk2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, lse2), x0, x1);
+                            float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                            if (cls == kDiag) {
+                                const int q0 = 64 * wg + 32 * qq + c;
+                                if (r > q0) p0 = 0.f;
+                                if (r > q0 + 1) p1 = 0.f;
+                            }
+                            const uint64_t pp = pk2(p0, p1);
+                            const uint64_t dd = mul2(pp, sub2(pk2(__uint_as_float(dpv[c]), __uint_as_float(dpv[c + 1])),
+                                                              hh ? pk2(Dl.z, Dl.w) : pk2(Dl.x, Dl.y)));
+                            float d0, d1;
+                            upk2(dd, d0, d1);
+                            pk[c >> 1] = pack_bf16x2(p0, p1);
+                            dsk[c >> 1] = pack_bf16x2(d0, d1);
                         }
-                        const float d0 = p0 * (__uint_as_float(dpv[c]) - del_s[q0]);
-                        const float d1 = p1 * (__uint_as_float(dpv[c + 1]) - del_s[q0 + 1]);
-                        pk[c >> 1] = pack_bf16x2(p0, p1);
-                        dsk[c >> 1] = pack_bf16x2(d0, d1);
                     }
                     tmem_st16(tS + 16 * qq, pk);
                     tmem_st16(tdP + 16 * qq, dsk);
@@ -574,17 +590,20 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
                 tmem_ld64(tS, sv);
                 tmem_ld64(tdP, dpv);
                 uint32_t dsk[32];
+                const uint64_t sl2x2 = pk2(sl2, sl2), nlse2 = pk2(-lse2, -lse2), del2 = pk2(delta, delta);
 #pragma unroll
                 for (int c = 0; c < 64; c += 2) {
                     const int k0 = 64 * wg + c;
-                    float p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lse2));
-                    float p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -lse2));
+                    float x0, x1;
+                    upk2(fma2(pk2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, nlse2), x0, x1);
+                    float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
                     if (cls == kDiag) {
                         if (k0 > r) p0 = 0.f;
                         if (k0 + 1 > r) p1 = 0.f;
                     }
-                    dsk[c >> 1] = pack_bf16x2(p0 * (__uint_as_float(dpv[c]) - delta),
-                                              p1 * (__uint_as_float(dpv[c + 1]) - delta));
+                    float d0, d1;
+                    upk2(mul2(pk2(p0, p1), sub2(pk2(__uint_as_float(dpv[c]), __uint_as_float(dpv[c + 1])), del2)), d0, d1);
+                    dsk[c >> 1] = pack_bf16x2(d0, d1);
                 }
                 tmem_st32(tdP, dsk);
                 tmem_wait_st();
