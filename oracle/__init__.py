@@ -46,14 +46,14 @@ def _L():
         lib.orc_rank_major_position.restype = i64
         lib.orc_rank_major_position.argtypes = [i64, i64, c_int, i64]
         lib.orc_attn_fwd_head.restype = None
-        lib.orc_attn_fwd_head.argtypes = [dp, dp, dp, i64, i64, c_int, c_double, ip, i64, dp, dp]
+        lib.orc_attn_fwd_head.argtypes = [dp, dp, dp, i64, i64, c_int, i64, c_double, ip, i64, dp, dp]
         lib.orc_ring_fwd_head.restype = None
-        lib.orc_ring_fwd_head.argtypes = [dp, dp, dp, i64, i64, c_int, c_double, i64, c_int,
+        lib.orc_ring_fwd_head.argtypes = [dp, dp, dp, i64, i64, c_int, i64, c_double, i64, c_int,
                                           ip, i64, dp, dp]
         lib.orc_lse_merge.restype = None
         lib.orc_lse_merge.argtypes = [dp, dp, dp, dp, i64, i64]
         lib.orc_attn_bwd_head.restype = None
-        lib.orc_attn_bwd_head.argtypes = [dp, dp, dp, dp, i64, i64, c_int, c_double,
+        lib.orc_attn_bwd_head.argtypes = [dp, dp, dp, dp, i64, i64, c_int, i64, c_double,
                                           ip, i64, dp, ip, i64, dp, dp]
         lib.orc_ring_owner.restype = i64
         lib.orc_ring_owner.argtypes = [i64, i64, i64]
@@ -163,8 +163,11 @@ def _rows_arg(rows, S):
     return _i64(np.arange(S) if rows is None else rows)
 
 
-def attn_fwd(q, k, v, causal: bool, scale: float = None, rows=None):
+def attn_fwd(q, k, v, causal: bool, scale: float = None, rows=None, window: int = 0):
     """Dense softmax attention in natural order.
+
+    window: with causal, each query sees its last `window` keys (itself
+    included); 0 = no window.
 
     q [B,H,S,D], k/v [B,Hkv,Sk,D] (numpy or torch, any float dtype; widened to
     fp64 one head at a time); query head h reads KV head h // (H/Hkv).
@@ -187,13 +190,14 @@ def attn_fwd(q, k, v, causal: bool, scale: float = None, rows=None):
                 qh = _f64(_rows_of(q[b, h], r) if rows is not None else q[b, h])
                 ob = np.zeros((len(r), D))
                 lb = np.zeros(len(r))
-                lib.orc_attn_fwd_head(_p(qh), _p(kh), _p(vh), Sk, D, int(causal), scale,
-                                      _p(r, ctypes.c_int64), len(r), _p(ob), _p(lb))
+                lib.orc_attn_fwd_head(_p(qh), _p(kh), _p(vh), Sk, D, int(causal), int(window),
+                                      scale, _p(r, ctypes.c_int64), len(r), _p(ob), _p(lb))
                 o[b, h], lse[b, h] = ob, lb
     return o, lse
 
 
-def ring_fwd(q, k, v, causal: bool, P: int, order: int, scale: float = None, rows=None):
+def ring_fwd(q, k, v, causal: bool, P: int, order: int, scale: float = None, rows=None,
+             window: int = 0):
     """Ring-structured forward: per (rank, step) partials merged step by step.
 
     Same arguments and results as attn_fwd (natural order in and out); the
@@ -214,8 +218,8 @@ def ring_fwd(q, k, v, causal: bool, P: int, order: int, scale: float = None, row
                 qh = _f64(_rows_of(q[b, h], r) if rows is not None else q[b, h])
                 ob = np.zeros((len(r), D))
                 lb = np.zeros(len(r))
-                lib.orc_ring_fwd_head(_p(qh), _p(kh), _p(vh), S, D, int(causal), scale, P,
-                                      order, _p(r, ctypes.c_int64), len(r), _p(ob), _p(lb))
+                lib.orc_ring_fwd_head(_p(qh), _p(kh), _p(vh), S, D, int(causal), int(window), scale,
+                                      P, order, _p(r, ctypes.c_int64), len(r), _p(ob), _p(lb))
                 o[b, h], lse[b, h] = ob, lb
     return o, lse
 
@@ -233,7 +237,7 @@ def lse_merge(o_acc, lse_acc, o_part, lse_part):
 
 
 def attn_bwd(q, k, v, dout, causal: bool, scale: float = None, qrows=None,
-             krows=None, heads=None):
+             krows=None, heads=None, window: int = 0):
     """Gradients of L = sum(dout * O) for dense attention (natural order).
 
     qrows: natural query positions for dQ (None = all); krows: key positions
@@ -269,8 +273,8 @@ def attn_bwd(q, k, v, dout, causal: bool, scale: float = None, qrows=None,
         dq = np.zeros((max(nq, 1), D))
         dk = np.zeros((max(nk, 1), D))
         dv = np.zeros((max(nk, 1), D))
-        lib.orc_attn_bwd_head(_p(qh), _p(kh), _p(vh), _p(doh), S, D, int(causal), scale,
-                              _p(qr, ctypes.c_int64), nq, _p(dq),
+        lib.orc_attn_bwd_head(_p(qh), _p(kh), _p(vh), _p(doh), S, D, int(causal), int(window),
+                              scale, _p(qr, ctypes.c_int64), nq, _p(dq),
                               _p(kr, ctypes.c_int64), nk, _p(dk), _p(dv))
         if want_q:
             dq_out[(b, h)] = dq[:nq]

@@ -12,6 +12,8 @@
  *     output together with its log-sum-exp);
  *   - causal masking: key j is visible to query i iff j <= i in GLOBAL token
  *     positions ("DeDLOC Guide", Best Practices table, Causal Mask Handling);
+ *     with a sliding window of W keys (axolotl-ringmaster README, Status:
+ *     sliding-window attention via flash's `window`), also j > i - W;
  *   - the merge of two partial (O, LSE) pairs by max-shifted exponential weights
  *     ("DeDLOC Guide", section 3 "Online Softmax Rescaling Across Decentralized
  *     Ranks", the alpha/beta equations, in the normalised-output form of Step 3);
@@ -84,6 +86,19 @@ static int rank_holds(int64_t S, int64_t P, int order, int64_t r, int64_t j)
 /* Dense attention of one head, the plain definition.                         */
 /* ------------------------------------------------------------------------- */
 
+/* Visible keys of the query at position i among S keys: [lo, hi).
+ * Non-causal: all. Causal: j <= i. Causal with a window of W > 0 keys:
+ * i - W < j <= i. */
+static void visible_range(int64_t i, int64_t S, int causal, int64_t window, int64_t* lo,
+                          int64_t* hi)
+{
+    *lo = 0;
+    *hi = S;
+    if (!causal) return;
+    *hi = i + 1 < S ? i + 1 : S;
+    if (window > 0 && i - window + 1 > 0) *lo = i - window + 1;
+}
+
 static double dot(const double* a, const double* b, int64_t D)
 {
     double acc = 0.0;
@@ -92,25 +107,27 @@ static double dot(const double* a, const double* b, int64_t D)
 }
 
 /* For query at natural position i over the visible key set
- * V(i) = {0..S-1} (non-causal) or {0..min(i, S-1)} (causal), S keys in k, v:
+ * V(i) = {0..S-1} (non-causal), {0..min(i, S-1)} (causal) or, with a window
+ * of W > 0 keys, {max(0, i-W+1)..min(i, S-1)}; S keys in k, v:
  *   LSE_i = m + ln sum_j exp(s_ij - m),  m = max_j s_ij
  *   O_i   = sum_j exp(s_ij - LSE_i) v_j
  * scratch must hold S doubles. */
 static void attend_row(const double* qi, const double* k, const double* v, int64_t S,
-                       int64_t D, int causal, double scale, int64_t i, double* s,
-                       double* o, double* lse)
+                       int64_t D, int causal, int64_t window, double scale, int64_t i,
+                       double* s, double* o, double* lse)
 {
-    int64_t n = (causal && i + 1 < S) ? i + 1 : S;
+    int64_t j0, n;
+    visible_range(i, S, causal, window, &j0, &n);
     double m = -INFINITY;
-    for (int64_t j = 0; j < n; ++j) {
+    for (int64_t j = j0; j < n; ++j) {
         s[j] = scale * dot(qi, k + j * D, D);
         if (s[j] > m) m = s[j];
     }
     double sum = 0.0;
-    for (int64_t j = 0; j < n; ++j) sum += exp(s[j] - m);
+    for (int64_t j = j0; j < n; ++j) sum += exp(s[j] - m);
     double L = m + log(sum);
     for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
-    for (int64_t j = 0; j < n; ++j) {
+    for (int64_t j = j0; j < n; ++j) {
         double p = exp(s[j] - L);
         const double* vj = v + j * D;
         for (int64_t d = 0; d < D; ++d) o[d] += p * vj[d];
@@ -122,15 +139,16 @@ static void attend_row(const double* qi, const double* k, const double* v, int64
  * position of q row r. k, v hold the Sk keys 0..Sk-1. Causal: the query at
  * position i sees keys j <= i. */
 void orc_attn_fwd_head(const double* q, const double* k, const double* v, int64_t Sk,
-                       int64_t D, int causal, double scale, const int64_t* rows,
-                       int64_t nrows, double* o, double* lse)
+                       int64_t D, int causal, int64_t window, double scale,
+                       const int64_t* rows, int64_t nrows, double* o, double* lse)
 {
 #pragma omp parallel
     {
         double* s = (double*)malloc(sizeof(double) * (size_t)Sk);
 #pragma omp for schedule(dynamic, 4)
         for (int64_t r = 0; r < nrows; ++r)
-            attend_row(q + r * D, k, v, Sk, D, causal, scale, rows[r], s, o + r * D, lse + r);
+            attend_row(q + r * D, k, v, Sk, D, causal, window, scale, rows[r], s, o + r * D,
+                       lse + r);
         free(s);
     }
 }
@@ -178,8 +196,8 @@ void orc_lse_merge(double* o_acc, double* lse_acc, const double* o_part,
  * order with merge_pair. The result equals the dense definition exactly up to
  * rounding, which the tests check. */
 void orc_ring_fwd_head(const double* q, const double* k, const double* v, int64_t S,
-                       int64_t D, int causal, double scale, int64_t P, int order,
-                       const int64_t* rows, int64_t nrows, double* o, double* lse)
+                       int64_t D, int causal, int64_t window, double scale, int64_t P,
+                       int order, const int64_t* rows, int64_t nrows, double* o, double* lse)
 {
 #pragma omp parallel
     {
@@ -189,6 +207,8 @@ void orc_ring_fwd_head(const double* q, const double* k, const double* v, int64_
         for (int64_t rr = 0; rr < nrows; ++rr) {
             int64_t x = rows[rr];
             int64_t i = rank_of_position(S, P, order, x);
+            int64_t jlo, jhi;
+            visible_range(x, S, causal, window, &jlo, &jhi);
             double* oacc = o + rr * D;
             double lacc = -INFINITY;
             for (int64_t d = 0; d < D; ++d) oacc[d] = 0.0;
@@ -197,7 +217,7 @@ void orc_ring_fwd_head(const double* q, const double* k, const double* v, int64_
                 /* partial over visible keys of owner r */
                 double m = -INFINITY;
                 for (int64_t j = 0; j < S; ++j) {
-                    if (!rank_holds(S, P, order, r, j) || (causal && j > x)) continue;
+                    if (!rank_holds(S, P, order, r, j) || j < jlo || j >= jhi) continue;
                     s[j] = scale * dot(q + rr * D, k + j * D, D);
                     if (s[j] > m) m = s[j];
                 }
@@ -206,12 +226,12 @@ void orc_ring_fwd_head(const double* q, const double* k, const double* v, int64_
                 if (m != -INFINITY) {
                     double sum = 0.0;
                     for (int64_t j = 0; j < S; ++j) {
-                        if (!rank_holds(S, P, order, r, j) || (causal && j > x)) continue;
+                        if (!rank_holds(S, P, order, r, j) || j < jlo || j >= jhi) continue;
                         sum += exp(s[j] - m);
                     }
                     lpart = m + log(sum);
                     for (int64_t j = 0; j < S; ++j) {
-                        if (!rank_holds(S, P, order, r, j) || (causal && j > x)) continue;
+                        if (!rank_holds(S, P, order, r, j) || j < jlo || j >= jhi) continue;
                         double p = exp(s[j] - lpart);
                         for (int64_t d = 0; d < D; ++d) op[d] += p * v[j * D + d];
                     }
@@ -238,8 +258,8 @@ void orc_ring_fwd_head(const double* q, const double* k, const double* v, int64_
  * (natural positions). For one head; a KV head shared by G query heads gets the
  * sum of its query heads' dK/dV, which the caller forms. */
 void orc_attn_bwd_head(const double* q, const double* k, const double* v,
-                       const double* dout, int64_t S, int64_t D, int causal, double scale,
-                       const int64_t* qrows, int64_t nq, double* dq,
+                       const double* dout, int64_t S, int64_t D, int causal, int64_t window,
+                       double scale, const int64_t* qrows, int64_t nq, double* dq,
                        const int64_t* krows, int64_t nk, double* dk, double* dv)
 {
     /* dQ rows: one forward row each, then the sum over its keys. */
@@ -251,12 +271,13 @@ void orc_attn_bwd_head(const double* q, const double* k, const double* v,
         for (int64_t r = 0; r < nq; ++r) {
             int64_t i = qrows[r];
             double L;
-            attend_row(q + i * D, k, v, S, D, causal, scale, i, s, oi, &L);
+            attend_row(q + i * D, k, v, S, D, causal, window, scale, i, s, oi, &L);
             double delta = dot(dout + i * D, oi, D);
-            int64_t n = causal ? i + 1 : S;
+            int64_t j0, n;
+            visible_range(i, S, causal, window, &j0, &n);
             double* g = dq + r * D;
             for (int64_t d = 0; d < D; ++d) g[d] = 0.0;
-            for (int64_t j = 0; j < n; ++j) {
+            for (int64_t j = j0; j < n; ++j) {
                 double p = exp(s[j] - L);
                 double ds = p * (dot(dout + i * D, v + j * D, D) - delta);
                 for (int64_t d = 0; d < D; ++d) g[d] += ds * k[j * D + d];
@@ -280,7 +301,7 @@ void orc_attn_bwd_head(const double* q, const double* k, const double* v,
         double* oi = (double*)malloc(sizeof(double) * (size_t)D);
 #pragma omp for schedule(dynamic, 16)
         for (int64_t i = i0; i < S; ++i) {
-            attend_row(q + i * D, k, v, S, D, causal, scale, i, s, oi, &lse_all[i]);
+            attend_row(q + i * D, k, v, S, D, causal, window, scale, i, s, oi, &lse_all[i]);
             delta_all[i] = dot(dout + i * D, oi, D);
         }
         free(oi);
@@ -292,8 +313,10 @@ void orc_attn_bwd_head(const double* q, const double* k, const double* v,
         double* gk = dk + r * D;
         double* gv = dv + r * D;
         for (int64_t d = 0; d < D; ++d) { gk[d] = 0.0; gv[d] = 0.0; }
+        /* query rows that see key j: i >= j (causal) and i < j + W (window) */
         int64_t ibeg = causal ? j : 0;
-        for (int64_t i = ibeg; i < S; ++i) {
+        int64_t iend = (causal && window > 0 && j + window < S) ? j + window : S;
+        for (int64_t i = ibeg; i < iend; ++i) {
             double sij = scale * dot(q + i * D, k + j * D, D);
             double p = exp(sij - lse_all[i]);
             double ds = p * (dot(dout + i * D, v + j * D, D) - delta_all[i]);

@@ -315,3 +315,121 @@ def test_ulysses_layout_is_a_bijection():
     for b, s, h, d in [(0, 0, 0, 0), (1, 11, 3, 2), (0, 5, 2, 1)]:
         assert dst[b, h, s, d] == src[b, s, h, d]
     assert np.array_equal(oracle.ulysses_head_to_seq(dst), src)
+
+
+# --- causal sliding window (axolotl-ringmaster README, Status: sliding-window
+# attention via flash's `window`): query i sees keys i-W < j <= i ---
+
+def _np_window_attention(q, k, v, W, scale):
+    """Band-masked dense attention with numpy/scipy (independent of the oracle)."""
+    B, H, S, D = q.shape
+    G = H // k.shape[1]
+    i = np.arange(S)[:, None]
+    j = np.arange(S)[None, :]
+    hidden = (j > i) | (j <= i - W)
+    o = np.zeros((B, H, S, D))
+    lse = np.zeros((B, H, S))
+    for b in range(B):
+        for h in range(H):
+            s = np.where(hidden, -np.inf, scale * q[b, h] @ k[b, h // G].T)
+            lse[b, h] = logsumexp(s, axis=-1)
+            o[b, h] = np.exp(s - lse[b, h][:, None]) @ v[b, h // G]
+    return o, lse
+
+
+@pytest.mark.parametrize("W", [1, 2, 3, 7, 16, 40])
+@pytest.mark.parametrize("H,Hkv,S,D", [(4, 2, 17, 5), (2, 2, 33, 8), (3, 1, 9, 3)])
+def test_window_forward_matches_numpy_bruteforce(W, H, Hkv, S, D):
+    seed = 7000 + W * 31 + S
+    q, k, v = _rand((2, H, S, D), seed), _rand((2, Hkv, S, D), seed + 1), _rand((2, Hkv, S, D), seed + 2)
+    scale = 1 / math.sqrt(D)
+    o, lse = oracle.attn_fwd(q, k, v, True, scale, window=W)
+    o_ref, lse_ref = _np_window_attention(q, k, v, W, scale)
+    np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=1e-13)
+
+
+def test_window_special_cases():
+    B, H, Hkv, S, D = 1, 4, 2, 23, 6
+    q, k, v = _rand((B, H, S, D), 71), _rand((B, Hkv, S, D), 72), _rand((B, Hkv, S, D), 73)
+    scale = 0.41
+    # W = 1: each query sees only its own key, so O_i = v_i and LSE_i = s_ii
+    o, lse = oracle.attn_fwd(q, k, v, True, scale, window=1)
+    kk = np.repeat(k, 2, axis=1)
+    np.testing.assert_allclose(o, np.repeat(v, 2, axis=1), atol=1e-14, rtol=0)
+    np.testing.assert_allclose(lse, scale * (q * kk).sum(-1), atol=1e-13, rtol=0)
+    # W >= S and W = 0 are plain causal attention; non-causal ignores W
+    o_c, lse_c = _np_attention(q, k, v, True, scale)
+    for W in (0, S, S + 5):
+        o_w, lse_w = oracle.attn_fwd(q, k, v, True, scale, window=W)
+        np.testing.assert_allclose(o_w, o_c, atol=1e-13, rtol=0)
+        np.testing.assert_allclose(lse_w, lse_c, atol=1e-13, rtol=0)
+    o_n, _ = oracle.attn_fwd(q, k, v, False, scale, window=3)
+    np.testing.assert_allclose(o_n, _np_attention(q, k, v, False, scale)[0], atol=1e-13, rtol=0)
+
+
+@pytest.mark.parametrize("order", [oracle.CONTIGUOUS, oracle.ZIGZAG])
+@pytest.mark.parametrize("P,W", [(2, 5), (3, 1), (4, 9), (4, 30), (5, 13)])
+def test_window_ring_equals_dense(order, P, W):
+    B, H, Hkv, D = 1, 2, 1, 4
+    S = 2 * P * 4
+    q, k, v = _rand((B, H, S, D), 80 + P), _rand((B, Hkv, S, D), 81 + P), _rand((B, Hkv, S, D), 82 + P)
+    o_ref, lse_ref = _np_window_attention(q, k, v, W, 0.5)
+    # natural order in and out; the ring layout decides each step's key subset
+    o, lse = oracle.ring_fwd(q, k, v, True, P, order, 0.5, window=W)
+    np.testing.assert_allclose(o, o_ref, atol=1e-13, rtol=0)
+    np.testing.assert_allclose(lse, lse_ref, atol=1e-13, rtol=0)
+
+
+@pytest.mark.parametrize("W", [1, 3, 8])
+def test_window_backward_matches_torch_autograd(W):
+    B, H, Hkv, S, D = 1, 4, 2, 14, 5
+    q, k, v = _rand((B, H, S, D), 90 + W), _rand((B, Hkv, S, D), 91 + W), _rand((B, Hkv, S, D), 92 + W)
+    dout = _rand((B, H, S, D), 93 + W)
+    scale = 0.45
+    tq, tk, tv = (torch.tensor(a, requires_grad=True) for a in (q, k, v))
+    kk = tk.repeat_interleave(H // Hkv, dim=1)
+    vv = tv.repeat_interleave(H // Hkv, dim=1)
+    i = torch.arange(S)[:, None]
+    j = torch.arange(S)[None, :]
+    s = (torch.matmul(tq, kk.transpose(-1, -2)) * scale).masked_fill((j > i) | (j <= i - W),
+                                                                     float("-inf"))
+    (torch.matmul(torch.softmax(s, -1), vv) * torch.tensor(dout)).sum().backward()
+    dq, dkv = oracle.attn_bwd(q, k, v, dout, True, scale, window=W)
+    for h in range(H):
+        np.testing.assert_allclose(dq[(0, h)], tq.grad[0, h].numpy(), atol=1e-12, rtol=0)
+    for g in range(Hkv):
+        np.testing.assert_allclose(dkv[(0, g)][0], tk.grad[0, g].numpy(), atol=1e-12, rtol=0)
+        np.testing.assert_allclose(dkv[(0, g)][1], tv.grad[0, g].numpy(), atol=1e-12, rtol=0)
+    if W == 1:
+        # O_i = v_i does not depend on q or k: dQ = dK = 0, dV_i = sum over the group of dO_i
+        assert max(np.abs(dq[(0, h)]).max() for h in range(H)) == 0
+        np.testing.assert_allclose(dkv[(0, 0)][1], dout[0, 0] + dout[0, 1], atol=1e-14)
+
+
+def test_window_backward_finite_differences_and_row_subsets():
+    B, H, Hkv, S, D, W = 1, 2, 1, 11, 3, 4
+    q, k, v = _rand((B, H, S, D), 95), _rand((B, Hkv, S, D), 96), _rand((B, Hkv, S, D), 97)
+    dout = _rand((B, H, S, D), 98)
+    dq, dkv = oracle.attn_bwd(q, k, v, dout, True, 0.6, window=W)
+
+    def loss(qq, kk_):
+        o, _ = oracle.attn_fwd(qq, kk_, v, True, 0.6, window=W)
+        return float((o * dout).sum())
+    h = 1e-6
+    for (s_, d_) in ((0, 0), (5, 2), (10, 1)):
+        qp, qm = q.copy(), q.copy()
+        qp[0, 1, s_, d_] += h
+        qm[0, 1, s_, d_] -= h
+        fd = (loss(qp, k) - loss(qm, k)) / (2 * h)
+        assert abs(fd - dq[(0, 1)][s_, d_]) <= 1e-7 * max(1.0, abs(fd))
+        kp, km = k.copy(), k.copy()
+        kp[0, 0, s_, d_] += h
+        km[0, 0, s_, d_] -= h
+        fd = (loss(q, kp) - loss(q, km)) / (2 * h)
+        assert abs(fd - dkv[(0, 0)][0][s_, d_]) <= 1e-7 * max(1.0, abs(fd))
+    rows = np.array([0, 4, 10])
+    dq_s, dkv_s = oracle.attn_bwd(q, k, v, dout, True, 0.6, qrows=rows, krows=rows,
+                                  heads=([(0, 0)], [(0, 0)]), window=W)
+    np.testing.assert_allclose(dq_s[(0, 0)], dq[(0, 0)][rows], atol=1e-13)
+    np.testing.assert_allclose(dkv_s[(0, 0)][0], dkv[(0, 0)][0][rows], atol=1e-13)
