@@ -98,6 +98,28 @@ RM_API rm_status rm_ring_attn_fwd(const void* q, const void* k, const void* v, v
                            rm_order order, rm_dtype dtype, float scale, cudaStream_t stream);
 
 /*
+ * rm_ring_attn_fwd_window — rm_ring_attn_fwd with a causal sliding window.
+ *
+ * The axolotl-ringmaster README's Status table (phase 4) lists sliding-window
+ * attention, passed to flash attention as its `window`. Here the window counts
+ * keys: query at global position i sees keys j with i - window < j <= i, that
+ * is itself and the window - 1 keys before it (flash's left window of
+ * window - 1, right window 0). Positions are global, as for the causal mask,
+ * so the result does not depend on P or the chunk order.
+ *
+ *   Arguments and layouts as rm_ring_attn_fwd, with the mask always causal.
+ *   window >= 1; window >= S gives plain causal attention. window < 1 returns
+ *   RM_ERR_INVALID_ARG; S >= 2^30 with a window below S returns
+ *   RM_ERR_UNSUPPORTED.
+ *   Key tiles outside every row's window are skipped, so the work grows with
+ *   S * window instead of S^2 / 2.
+ */
+RM_API rm_status rm_ring_attn_fwd_window(const void* q, const void* k, const void* v, void* o,
+                                         float* lse, int B, int H, int Hkv, int S, int D, int P,
+                                         int window, rm_order order, rm_dtype dtype, float scale,
+                                         cudaStream_t stream);
+
+/*
  * rm_ring_attn_bwd — gradients of L = sum(dO * O) through the ring forward
  * (axolotl-ringmaster README: flash-style reverse-ring backward; gradients
  * accumulate in fp32 across ring steps).
@@ -124,6 +146,20 @@ RM_API rm_status rm_ring_attn_bwd(const void* q, const void* k, const void* v, c
                            float* dv, void* workspace, size_t workspace_bytes, int B, int H,
                            int Hkv, int S, int D, int P, int causal, rm_order order,
                            rm_dtype dtype, float scale, cudaStream_t stream);
+
+/*
+ * rm_ring_attn_bwd_window — rm_ring_attn_bwd through rm_ring_attn_fwd_window:
+ * the same gradients with P_ij = 0 outside the window (query i, keys
+ * i - window < j <= i). Arguments, layouts, workspace, outputs and status codes
+ * as rm_ring_attn_bwd; window rules as rm_ring_attn_fwd_window. o and lse must
+ * come from the windowed forward with the same window.
+ */
+RM_API rm_status rm_ring_attn_bwd_window(const void* q, const void* k, const void* v,
+                                         const void* o, const float* lse, const void* dout,
+                                         float* dq, float* dk, float* dv, void* workspace,
+                                         size_t workspace_bytes, int B, int H, int Hkv, int S,
+                                         int D, int P, int window, rm_order order,
+                                         rm_dtype dtype, float scale, cudaStream_t stream);
 
 /*
  * rm_ring_attn_bwd_noalloc — rm_ring_attn_bwd for callers that cannot allocate.

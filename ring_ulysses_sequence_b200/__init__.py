@@ -41,9 +41,10 @@ def _need(t, name):
 
 
 def ring_attn_fwd(q, k, v, P, causal=True, order="zigzag", scale=None, out=None, lse=None,
-                  stream=None):
+                  stream=None, window=0):
     """Ring attention forward. q [B,H,S,D], k/v [B,Hkv,S,D] (rank-major S).
 
+    window > 0 (causal only): query i sees keys i - window < j <= i.
     Returns (O [B,H,S,D] in q's dtype, LSE [B,H,S] float32).
     """
     import torch
@@ -56,14 +57,23 @@ def ring_attn_fwd(q, k, v, P, causal=True, order="zigzag", scale=None, out=None,
     if lse is None:
         lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
-    native.rm_ring_attn_fwd(q, k, v, out, lse, B, H, Hkv, S, D, P, causal, _order(order),
-                            _dtype_code(q), scale, stream)
+    if window:
+        if not causal:
+            raise ValueError("a sliding window needs causal=True")
+        native.rm_ring_attn_fwd_window(q, k, v, out, lse, B, H, Hkv, S, D, P, window,
+                                       _order(order), _dtype_code(q), scale, stream)
+    else:
+        native.rm_ring_attn_fwd(q, k, v, out, lse, B, H, Hkv, S, D, P, causal, _order(order),
+                                _dtype_code(q), scale, stream)
     return out, lse
 
 
 def ring_attn_bwd(q, k, v, o, lse, dout, P, causal=True, order="zigzag", scale=None,
-                  workspace=None, stream=None):
-    """Ring attention backward. Returns fp32 (dQ, dK, dV)."""
+                  workspace=None, stream=None, window=0):
+    """Ring attention backward. Returns fp32 (dQ, dK, dV).
+
+    window: as in ring_attn_fwd (o and lse must come from that window).
+    """
     import torch
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (lse, "lse"), (dout, "dout")):
         _need(t, n)
@@ -76,9 +86,16 @@ def ring_attn_bwd(q, k, v, o, lse, dout, P, causal=True, order="zigzag", scale=N
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
-    native.rm_ring_attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace.numel(),
-                            B, H, Hkv, S, D, P, causal, _order(order), _dtype_code(q), scale,
-                            stream)
+    if window:
+        if not causal:
+            raise ValueError("a sliding window needs causal=True")
+        native.rm_ring_attn_bwd_window(q, k, v, o, lse, dout, dq, dk, dv, workspace,
+                                       workspace.numel(), B, H, Hkv, S, D, P, window,
+                                       _order(order), _dtype_code(q), scale, stream)
+    else:
+        native.rm_ring_attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace.numel(),
+                                B, H, Hkv, S, D, P, causal, _order(order), _dtype_code(q), scale,
+                                stream)
     return dq, dk, dv
 
 

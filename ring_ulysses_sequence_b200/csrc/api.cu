@@ -104,6 +104,43 @@ static rm_status check_attn(const void* q, const void* k, const void* v, int B, 
     return RM_OK;
 }
 
+// Window argument of the *_window entry points -> AttnShape::window: a window
+// that covers the whole sequence is plain causal attention (0).
+static rm_status window_arg(int window, int S, int* out) {
+    if (window < 1) return RM_ERR_INVALID_ARG;
+    *out = window >= S ? 0 : window;
+    // the tile iterators add window and position in int arithmetic
+    if (*out && S >= (1 << 30)) return RM_ERR_UNSUPPORTED;
+    return RM_OK;
+}
+
+static rm_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int H, int Hkv, int S, int D, int P, int causal, int window,
+                          rm_order order, rm_dtype dtype, float scale, cudaStream_t stream) {
+    const int tile_q = dtype == RM_DTYPE_BF16 ? 128 : 64;
+    rm_status st = check_attn(q, k, v, B, H, Hkv, S, D, P, order, dtype, scale, tile_q);
+    if (st != RM_OK) return st;
+    if (B == 0 || S == 0) return RM_OK;  // empty batch or sequence: nothing to do
+    if (!o || !lse || !aligned16(o) || !aligned16(lse)) return RM_ERR_INVALID_ARG;
+    LaunchCtx ctx;
+    if ((st = get_ctx(stream, &ctx)) != RM_OK) return st;
+    AttnShape sh{B, H, Hkv, S, D, P, causal ? 1 : 0, order == RM_ORDER_ZIGZAG ? 1 : 0, scale,
+                 window};
+    cudaError_t e = dtype == RM_DTYPE_BF16
+                        ? launch_fwd_tc(sh, q, k, v, o, lse, ctx)
+                        : launch_fwd_fp32(sh, static_cast<const float*>(q),
+                                          static_cast<const float*>(k),
+                                          static_cast<const float*>(v), static_cast<float*>(o),
+                                          lse, ctx);
+    return e == cudaSuccess ? RM_OK : cuda_fail(e);
+}
+
+static rm_status bwd_impl(const void* q, const void* k, const void* v, const void* o,
+                          const float* lse, const void* dout, float* dq, float* dk, float* dv,
+                          void* workspace, size_t workspace_bytes, int B, int H, int Hkv, int S,
+                          int D, int P, int causal, int window, rm_order order, rm_dtype dtype,
+                          float scale, cudaStream_t stream);
+
 }  // namespace rm
 
 using namespace rm;
@@ -155,21 +192,17 @@ rm_status rm_watchdog_selftest(uint64_t timeout_ns, cudaStream_t stream) {
 rm_status rm_ring_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                            int B, int H, int Hkv, int S, int D, int P, int causal,
                            rm_order order, rm_dtype dtype, float scale, cudaStream_t stream) {
-    const int tile_q = dtype == RM_DTYPE_BF16 ? 128 : 64;
-    rm_status st = check_attn(q, k, v, B, H, Hkv, S, D, P, order, dtype, scale, tile_q);
+    return fwd_impl(q, k, v, o, lse, B, H, Hkv, S, D, P, causal, 0, order, dtype, scale, stream);
+}
+
+rm_status rm_ring_attn_fwd_window(const void* q, const void* k, const void* v, void* o,
+                                  float* lse, int B, int H, int Hkv, int S, int D, int P,
+                                  int window, rm_order order, rm_dtype dtype, float scale,
+                                  cudaStream_t stream) {
+    int w = 0;
+    rm_status st = window_arg(window, S, &w);
     if (st != RM_OK) return st;
-    if (B == 0 || S == 0) return RM_OK;  // empty batch or sequence: nothing to do
-    if (!o || !lse || !aligned16(o) || !aligned16(lse)) return RM_ERR_INVALID_ARG;
-    LaunchCtx ctx;
-    if ((st = get_ctx(stream, &ctx)) != RM_OK) return st;
-    AttnShape sh{B, H, Hkv, S, D, P, causal ? 1 : 0, order == RM_ORDER_ZIGZAG ? 1 : 0, scale};
-    cudaError_t e = dtype == RM_DTYPE_BF16
-                        ? launch_fwd_tc(sh, q, k, v, o, lse, ctx)
-                        : launch_fwd_fp32(sh, static_cast<const float*>(q),
-                                          static_cast<const float*>(k),
-                                          static_cast<const float*>(v), static_cast<float*>(o),
-                                          lse, ctx);
-    return e == cudaSuccess ? RM_OK : cuda_fail(e);
+    return fwd_impl(q, k, v, o, lse, B, H, Hkv, S, D, P, 1, w, order, dtype, scale, stream);
 }
 
 size_t rm_ring_attn_bwd_workspace_size(int B, int H, int S) {
@@ -183,6 +216,31 @@ rm_status rm_ring_attn_bwd(const void* q, const void* k, const void* v, const vo
                            void* workspace, size_t workspace_bytes, int B, int H, int Hkv,
                            int S, int D, int P, int causal, rm_order order, rm_dtype dtype,
                            float scale, cudaStream_t stream) {
+    return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv, S, D,
+                    P, causal, 0, order, dtype, scale, stream);
+}
+
+rm_status rm_ring_attn_bwd_window(const void* q, const void* k, const void* v, const void* o,
+                                  const float* lse, const void* dout, float* dq, float* dk,
+                                  float* dv, void* workspace, size_t workspace_bytes, int B,
+                                  int H, int Hkv, int S, int D, int P, int window, rm_order order,
+                                  rm_dtype dtype, float scale, cudaStream_t stream) {
+    int w = 0;
+    rm_status st = window_arg(window, S, &w);
+    if (st != RM_OK) return st;
+    return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv, S, D,
+                    P, 1, w, order, dtype, scale, stream);
+}
+
+}  // extern "C"
+
+namespace rm {
+
+static rm_status bwd_impl(const void* q, const void* k, const void* v, const void* o,
+                          const float* lse, const void* dout, float* dq, float* dk, float* dv,
+                          void* workspace, size_t workspace_bytes, int B, int H, int Hkv, int S,
+                          int D, int P, int causal, int window, rm_order order, rm_dtype dtype,
+                          float scale, cudaStream_t stream) {
     rm_status st = check_attn(q, k, v, B, H, Hkv, S, D, P, order, dtype, scale, 128);
     if (st != RM_OK) return st;
     if (dtype != RM_DTYPE_BF16) return RM_ERR_UNSUPPORTED;
@@ -194,11 +252,16 @@ rm_status rm_ring_attn_bwd(const void* q, const void* k, const void* v, const vo
     if (workspace_bytes < rm_ring_attn_bwd_workspace_size(B, H, S)) return RM_ERR_INVALID_ARG;
     LaunchCtx ctx;
     if ((st = get_ctx(stream, &ctx)) != RM_OK) return st;
-    AttnShape sh{B, H, Hkv, S, D, P, causal ? 1 : 0, order == RM_ORDER_ZIGZAG ? 1 : 0, scale};
+    AttnShape sh{B, H, Hkv, S, D, P, causal ? 1 : 0, order == RM_ORDER_ZIGZAG ? 1 : 0, scale,
+                 window};
     cudaError_t e = launch_bwd(sh, q, k, v, o, lse, dout, dq, dk, dv,
                                static_cast<float*>(workspace), ctx);
     return e == cudaSuccess ? RM_OK : cuda_fail(e);
 }
+
+}  // namespace rm
+
+extern "C" {
 
 rm_status rm_ring_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                                    const float* lse, const void* dout, float* dq, float* dk,

@@ -56,12 +56,6 @@ struct BCfg {
     static constexpr int kSmemQ = kQBarOff + 256 + 1024;
 };
 
-enum : int { kSkip = 0, kDiag = 1, kFull = 2 };
-__device__ __forceinline__ int tile_class(int causal, int qpos, int kpos) {
-    if (!causal) return kFull;
-    return kpos > qpos ? kSkip : (kpos == qpos ? kDiag : kFull);
-}
-
 // TMEM column of K-step k (16 elements) of a bf16 operand written by the two
 // compute warpgroups: warpgroup w packs its 64 columns into [64w, 64w+32).
 __device__ __forceinline__ uint32_t packed_col(int k) { return k < 4 ? 8 * k : 64 + 8 * (k - 4); }
@@ -76,6 +70,8 @@ struct BwdArgs {
     unsigned* status;
     unsigned long long timeout_ns;
     int B, H, Hkv, S, P, causal, G, n_items;
+    int window;      // causal left window in keys; 0 = none
+    unsigned band;   // window, or 2^31 - 1 without one: the visible width of a row
     float scale, scale_log2;
     RingLayout lay;
 };
@@ -111,14 +107,15 @@ __device__ __forceinline__ KvItem decode_kv_item(const BwdArgs& a, int w) {
 // Query tiles (head, slot, class) that see a key tile, in reverse-ring order:
 // step t visits rank (r + t) mod P; heads of the group innermost. A rank's
 // block is one (contiguous) or two (zigzag) runs of consecutive positions, and
-// the query tiles that see a causal key tile form a suffix of each run: O(1)
-// work per returned tile, no division.
+// the query tiles that see a causal key tile form a suffix of each run (with a
+// window, an interval of it): O(1) work per returned tile, no division. qpos
+// holds the natural position of the query tile last returned.
 struct QIter {
     const BwdArgs* a;
-    int rank, kpos, g, t, run, u, u_end, s0, p0, hh, cls, qslot;
+    int rank, kpos, g, t, run, u, u_end, s0, p0, hh, cls, qslot, qpos;
     __device__ __forceinline__ QIter(const BwdArgs& args, const KvItem& it)
         : a(&args), rank(it.rank), kpos(it.kpos), g(it.g), t(0), run(-1), u(0), u_end(0), s0(0),
-          p0(0), hh(args.G), cls(kSkip), qslot(0) {}
+          p0(0), hh(args.G), cls(kSkip), qslot(0), qpos(0) {}
     __device__ __forceinline__ bool next(int& h, int& slot, int& c) {
         const RingLayout& lay = a->lay;
         for (;;) {
@@ -141,9 +138,14 @@ struct QIter {
                 p0 = lay.zigzag ? (run == 0 ? i * lay.c : (2 * lay.P - 1 - i) * lay.c) : i * lay.L;
                 u_end = ctiles;
                 u = a->causal ? min(ctiles, max((kpos - p0) >> 7, 0)) : 0;  // first tile at or after the key
+                // window: the last query tile whose first row still sees the
+                // key tile's last key, qp <= kpos + 127 + W - 1
+                if (a->causal && a->window)
+                    u_end = min(ctiles, max(((kpos + a->window + (kT - 2) - p0) >> 7) + 1, 0));
             }
             qslot = s0 + u * kT;
-            cls = tile_class(a->causal, p0 + u * kT, kpos);
+            qpos = p0 + u * kT;
+            cls = band_tile_class(a->causal, a->window, qpos - kpos);
             ++u;
             hh = 0;
         }
@@ -328,6 +330,8 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
             while (ok && qi.next(h, qslot, cls)) {
                 const int st = uses % kStages;
                 ++uses;
+                // key row r sees query column c iff 0 <= c - lo < band
+                const int lo = r - (qi.qpos - it.kpos);
                 const float* lse_s = reinterpret_cast<const float*>(
                     smem + 2 * BCfg<D>::kTile + st * BCfg<D>::kStageKV + 2 * BCfg<D>::kTile);
                 const float* del_s = lse_s + kT;
@@ -358,10 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
                             float x0, x1;
                             upk2(fma2(pk2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, lse2), x0, x1);
                             float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                            if (cls == kDiag) {
+                            if (cls == kMask) {
                                 const int q0 = 64 * wg + 32 * qq + c;
-                                if (r > q0) p0 = 0.f;
-                                if (r > q0 + 1) p1 = 0.f;
+                                if (static_cast<unsigned>(q0 - lo) >= a.band) p0 = 0.f;
+                                if (static_cast<unsigned>(q0 + 1 - lo) >= a.band) p1 = 0.f;
                             }
                             const uint64_t pp = pk2(p0, p1);
                             const uint64_t dd = mul2(pp, sub2(pk2(__uint_as_float(dpv[c]), __uint_as_float(dpv[c + 1])),
@@ -418,12 +422,15 @@ __device__ __forceinline__ QItem decode_q_item(const BwdArgs& a, int w) {
 }
 
 // Key tiles a query tile sees, in ring order: step t visits owner (i - t) mod P;
-// within each run of an owner's block the visible tiles are a prefix.
+// within each run of an owner's block the visible tiles are a prefix (with a
+// window, an interval). kpos holds the natural position of the tile last
+// returned.
 struct KIter {
     const BwdArgs* a;
-    int rank, qpos, t, run, u, u_end, s0, p0;
+    int rank, qpos, t, run, u, u_end, s0, p0, kpos;
     __device__ __forceinline__ KIter(const BwdArgs& args, const QItem& it)
-        : a(&args), rank(it.rank), qpos(it.pos), t(0), run(-1), u(0), u_end(0), s0(0), p0(0) {}
+        : a(&args), rank(it.rank), qpos(it.pos), t(0), run(-1), u(0), u_end(0), s0(0), p0(0),
+          kpos(0) {}
     __device__ __forceinline__ bool next(int& kslot, int& cls) {
         const RingLayout& lay = a->lay;
         while (u >= u_end) {
@@ -438,9 +445,12 @@ struct KIter {
             p0 = lay.zigzag ? (run == 0 ? r * lay.c : (2 * lay.P - 1 - r) * lay.c) : r * lay.L;
             u = 0;
             u_end = a->causal ? min(ctiles, max(((qpos - p0) >> 7) + 1, 0)) : ctiles;
+            // window: the first tile whose last key is inside row 0's window
+            if (a->causal && a->window) u = max(0, ceil_div128(qpos - a->window - (kT - 2) - p0));
         }
         kslot = s0 + u * kT;
-        cls = tile_class(a->causal, qpos, p0 + u * kT);
+        kpos = p0 + u * kT;
+        cls = band_tile_class(a->causal, a->window, qpos - kpos);
         ++u;
         return true;
     }
@@ -583,6 +593,8 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
             KIter ki(a, it);
             int kslot, cls;
             while (ok && ki.next(kslot, cls)) {
+                // query row r sees key column c iff 0 <= hi - c < band
+                const int hi = r + it.pos - ki.kpos;
                 ok = mbar_wait(smem_u32(&bars.s_full), (s_cnt++) & 1, wd);
                 if (!ok) break;
                 tc_fence_after();
@@ -597,9 +609,9 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
                     float x0, x1;
                     upk2(fma2(pk2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, nlse2), x0, x1);
                     float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                    if (cls == kDiag) {
-                        if (k0 > r) p0 = 0.f;
-                        if (k0 + 1 > r) p1 = 0.f;
+                    if (cls == kMask) {
+                        if (static_cast<unsigned>(hi - k0) >= a.band) p0 = 0.f;
+                        if (static_cast<unsigned>(hi - k0 - 1) >= a.band) p1 = 0.f;
                     }
                     float d0, d1;
                     upk2(mul2(pk2(p0, p1), sub2(pk2(__uint_as_float(dpv[c]), __uint_as_float(dpv[c + 1])), del2)), d0, d1);
@@ -715,6 +727,8 @@ cudaError_t launch_bwd(const AttnShape& sh, const void* q, const void* k, const 
     a.P = sh.P;
     a.causal = sh.causal;
     a.G = sh.H / sh.Hkv;
+    a.window = sh.causal ? sh.window : 0;
+    a.band = a.window ? static_cast<unsigned>(a.window) : 0x7fffffffu;
     a.scale = sh.scale;
     a.scale_log2 = sh.scale * kLog2e;
     a.lay = RingLayout{sh.S, sh.P, sh.S / sh.P, sh.zigzag ? sh.S / (2 * sh.P) : sh.S / sh.P, sh.zigzag};

@@ -39,6 +39,24 @@ struct RingLayout {
     }
 };
 
+// Class of a (128-query tile, 128-key tile) pair from d = qpos - kpos, the
+// difference of the tiles' first natural positions (a multiple of 128). The
+// mask is causal ("DeDLOC Guide", Best Practices, Causal Mask Handling) with an
+// optional left window of W keys (axolotl-ringmaster README, Status:
+// sliding-window attention): query i sees keys i - W < j <= i; W = 0 means no
+// window. kSkip: no pair visible; kFull: every pair visible; kMask: mixed.
+enum : int { kSkip = 0, kMask = 1, kFull = 2 };
+__host__ __device__ __forceinline__ int band_tile_class(int causal, int window, int d) {
+    if (!causal) return kFull;
+    if (d < 0) return kSkip;                        // every key after every query
+    if (window == 0) return d == 0 ? kMask : kFull;
+    if (d >= window + 127) return kSkip;            // every key left of every window
+    return (d >= 128 && d <= window - 128) ? kFull : kMask;
+}
+
+// ceil(x / 128) for any sign of x (the shift rounds toward minus infinity).
+__host__ __device__ __forceinline__ int ceil_div128(int x) { return -((-x) >> 7); }
+
 // ---------------------------------------------------------------------------
 // Watchdog: every spin-wait is bounded in time.
 // ---------------------------------------------------------------------------

@@ -63,6 +63,8 @@ struct TcArgs {
     unsigned* status;
     unsigned long long timeout_ns;
     int H, Hkv, S, P, causal, G;
+    int window;        // causal left window in keys; 0 = none
+    unsigned band;     // window, or 2^31 - 1 without one: the visible width of a row
     int head_pair;     // 1: tiles are heads (h, h+1) at one slot; 0: one head, slots s, s+128
     int n_units;       // query units per head unit
     int n_head_units;  // B * (head_pair ? H / 2 : H)
@@ -103,25 +105,18 @@ __device__ __forceinline__ Item decode_item(const TcArgs& a, int w) {
     return it;
 }
 
-// Causal class of a (query tile, key tile) pair; both start on multiples of
-// 128 in natural positions (chunks are multiples of 128 tokens).
-enum : int { kSkip = 0, kDiag = 1, kFull = 2 };
-__device__ __forceinline__ int tile_class(int causal, int qpos, int kpos) {
-    if (!causal) return kFull;
-    return kpos > qpos ? kSkip : (kpos == qpos ? kDiag : kFull);
-}
-
 // Key tiles of an item in ring order: step t visits owner (rank - t) mod P.
 // An owner's block is one run (contiguous order) or two runs (zigzag: chunk r
 // then chunk 2P-1-r) of consecutive natural positions, so the tiles a causal
-// query tile can see form a prefix of each run: O(1) work per tile returned,
-// no division.
+// query tile can see form a prefix of each run, and with a window an interval
+// of it: O(1) work per tile returned, no division. kpos holds the natural
+// position of the tile last returned.
 struct KvIter {
     const TcArgs* a;   // layout read from the kernel parameters, not copied
-    int rank, pos0, pos1, t, run, u, u_end, s0, p0;
+    int rank, pos0, pos1, t, run, u, u_end, s0, p0, kpos;
     __device__ __forceinline__ KvIter(const TcArgs& args, const Item& it)
         : a(&args), rank(it.rank), pos0(it.pos0), pos1(it.pos1), t(0), run(-1), u(0), u_end(0),
-          s0(0), p0(0) {}
+          s0(0), p0(0), kpos(0) {}
     __device__ __forceinline__ bool next(int& kslot, int& c0, int& c1) {
         const RingLayout& lay = a->lay;
         while (u >= u_end) {
@@ -139,13 +134,16 @@ struct KvIter {
             if (a->causal) {
                 const int vis = ((max(pos0, pos1) - p0) >> 7) + 1;  // tiles at or before the query
                 u_end = min(ctiles, max(vis, 0));
+                // window: the first tile whose last key is inside the earliest
+                // row's window, kp + 127 > min(pos) - W
+                if (a->window) u = max(0, ceil_div128(min(pos0, pos1) - a->window - (kBN - 2) - p0));
             }
         }
-        const int kp = p0 + u * kBN;
+        kpos = p0 + u * kBN;
         kslot = s0 + u * kBN;
         ++u;
-        c0 = tile_class(a->causal, pos0, kp);
-        c1 = tile_class(a->causal, pos1, kp);
+        c0 = band_tile_class(a->causal, a->window, pos0 - kpos);
+        c1 = band_tile_class(a->causal, a->window, pos1 - kpos);
         return true;
     }
 };
@@ -372,10 +370,12 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
                     tmem_ld64(tS + 64, raw);
 #pragma unroll
                     for (int c = 0; c < 64; ++c) s[64 + c] = __uint_as_float(raw[c]);
-                    if (cls == kDiag) {
+                    if (cls == kMask) {
+                        // key column c is visible iff 0 <= hi - c < band
+                        const int hi = r + (x ? it.pos1 : it.pos0) - kv.kpos;
 #pragma unroll
                         for (int c = 0; c < 128; ++c)
-                            if (c > r) s[c] = -INFINITY;
+                            if (static_cast<unsigned>(hi - c) >= a.band) s[c] = -INFINITY;
                     }
                     float mx = s[0];
 #pragma unroll
@@ -389,7 +389,8 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
                         m = m_new;
                         rescale_o = j > 0;
                     }
-                    const float neg = -m * sl2;  // m is finite after a visible tile
+                    // m stays -inf while a windowed row has seen no key: p = 0 then
+                    const float neg = m == -INFINITY ? 0.f : -m * sl2;
                     float rs = 0.f;
                     uint32_t pk[32];
 #pragma unroll
@@ -479,6 +480,8 @@ cudaError_t launch_fwd_tc(const AttnShape& sh, const void* q, const void* k, con
     a.P = sh.P;
     a.causal = sh.causal;
     a.G = sh.H / sh.Hkv;
+    a.window = sh.causal ? sh.window : 0;
+    a.band = a.window ? static_cast<unsigned>(a.window) : 0x7fffffffu;
     a.head_pair = (a.G % 2 == 0) ? 1 : 0;
     a.n_units = a.head_pair ? sh.S / kBM : sh.S / (2 * kBM);
     a.n_head_units = sh.B * (a.head_pair ? sh.H / 2 : sh.H);

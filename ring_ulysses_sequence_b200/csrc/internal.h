@@ -19,6 +19,7 @@ struct LaunchCtx {
 struct AttnShape {
     int B, H, Hkv, S, D, P, causal, zigzag;
     float scale;
+    int window;  // causal left window in keys (query i sees i - window < j <= i); 0 = none
 };
 
 // Forward, bf16, tcgen05 tensor cores (fwd_tc.cu).

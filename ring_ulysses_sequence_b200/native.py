@@ -21,9 +21,13 @@ _vp, _i, _i64, _f, _sz, _u64 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, c
                                  ctypes.c_size_t, ctypes.c_uint64)
 SIGNATURES = {
     "rm_ring_attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
+    "rm_ring_attn_fwd_window": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i,
+                                     _f, _vp]),
     "rm_ring_attn_bwd_workspace_size": (_sz, [_i, _i, _i]),
     "rm_ring_attn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                               _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
+    "rm_ring_attn_bwd_window": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                                     _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "rm_ring_attn_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                       _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "rm_lse_merge": (_i, [_vp, _vp, _vp, _vp, _i64, _i, _vp]),
@@ -98,6 +102,12 @@ def rm_ring_attn_fwd(q, k, v, o, lse, B, H, Hkv, S, D, P, causal, order, dtype, 
                  int(causal), order, dtype, scale, _s(stream))
 
 
+def rm_ring_attn_fwd_window(q, k, v, o, lse, B, H, Hkv, S, D, P, window, order, dtype, scale,
+                            stream=None):
+    return _call("rm_ring_attn_fwd_window", _p(q), _p(k), _p(v), _p(o), _p(lse), B, H, Hkv, S, D,
+                 P, window, order, dtype, scale, _s(stream))
+
+
 def rm_ring_attn_bwd_workspace_size(B, H, S):
     return int(lib().rm_ring_attn_bwd_workspace_size(B, H, S))
 
@@ -107,6 +117,13 @@ def rm_ring_attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_byt
     return _call("rm_ring_attn_bwd", _p(q), _p(k), _p(v), _p(o), _p(lse), _p(dout), _p(dq),
                  _p(dk), _p(dv), _p(workspace), workspace_bytes, B, H, Hkv, S, D, P, int(causal),
                  order, dtype, scale, _s(stream))
+
+
+def rm_ring_attn_bwd_window(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H,
+                            Hkv, S, D, P, window, order, dtype, scale, stream=None):
+    return _call("rm_ring_attn_bwd_window", _p(q), _p(k), _p(v), _p(o), _p(lse), _p(dout),
+                 _p(dq), _p(dk), _p(dv), _p(workspace), workspace_bytes, B, H, Hkv, S, D, P,
+                 window, order, dtype, scale, _s(stream))
 
 
 def rm_ring_attn_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, H, Hkv, S, D, P, causal,

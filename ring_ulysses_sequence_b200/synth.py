@@ -32,6 +32,7 @@ class Workload:
     input_scale: float = 1.0
     ulysses: int = 1      # U; the ring size is P
     backward: bool = False
+    window: int = 0       # causal sliding window in keys (query i sees i-W < j <= i); 0 = none
     notes: str = field(default="", compare=False)
 
     @property
@@ -44,7 +45,12 @@ class Workload:
         return self.S // (2 * self.P) if self.order == "zigzag" else self.S // self.P
 
     def fwd_flops(self) -> float:
-        """Algorithmic forward FLOPs: 4 B H S^2 D, halved when causal."""
+        """Algorithmic forward FLOPs: 4 B H S^2 D, halved when causal; with a
+        window, 4 B H D times the number of visible (query, key) pairs."""
+        if self.causal and 0 < self.window < self.S:
+            W, S = self.window, self.S
+            pairs = W * (W + 1) // 2 + (S - W) * W
+            return 4.0 * self.B * self.H * self.D * pairs
         f = 4.0 * self.B * self.H * self.S * self.S * self.D
         return f / 2 if self.causal else f
 
@@ -66,6 +72,11 @@ WORKLOADS = {
     "ring_fwd_bf16_S32k_gqa_causal_zigzag": Workload("ring_fwd_bf16_S32k_gqa_causal_zigzag",
                                                      1, 32, 8, 32768, 128, 8, "zigzag", True,
                                                      torch.bfloat16, 2, 0.5),
+    # The same layer with a 4096-token causal sliding window (Mistral-style
+    # local attention): most key tiles of a query tile are skipped.
+    "ring_fwd_bf16_S32k_gqa_causal_zigzag_window4k": Workload(
+        "ring_fwd_bf16_S32k_gqa_causal_zigzag_window4k", 1, 32, 8, 32768, 128, 8, "zigzag", True,
+        torch.bfloat16, 5, 0.5, window=4096),
     # Ulysses x Ring: 4 x 4 mesh over 131072 tokens, sequence-sharded input
     # [16 shards, 8192 tokens, heads, 128].
     "usp_fwd_bf16_S128k_u4r4": Workload("usp_fwd_bf16_S128k_u4r4", 1, 32, 8, 131072, 128, 4,

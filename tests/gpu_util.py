@@ -39,13 +39,13 @@ def assert_close(got, ref, max_abs, mean_abs=None, what=""):
     return mx
 
 
-def run_fwd(qn, kn, vn, P, order, causal, scale=None):
+def run_fwd(qn, kn, vn, P, order, causal, scale=None, window=0):
     """Natural-order CPU inputs -> GPU ring forward -> natural-order CPU (O, LSE)."""
     import ring_ulysses_sequence_b200 as rm
     q = to_rank_major(qn, P, order).cuda()
     k = to_rank_major(kn, P, order).cuda()
     v = to_rank_major(vn, P, order).cuda()
-    o, lse = rm.ring_attn_fwd(q, k, v, P, causal=causal, order=order, scale=scale)
+    o, lse = rm.ring_attn_fwd(q, k, v, P, causal=causal, order=order, scale=scale, window=window)
     torch.cuda.synchronize()
     assert rm.native.rm_check_device_status() == 0
     return (to_natural(o.float().cpu(), P, order),

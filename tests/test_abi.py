@@ -28,6 +28,7 @@ def header_functions():
 def test_header_declares_the_path():
     fns = header_functions()
     for name in ("rm_ring_attn_fwd", "rm_ring_attn_bwd", "rm_ring_attn_bwd_workspace_size",
+                 "rm_ring_attn_fwd_window", "rm_ring_attn_bwd_window",
                  "rm_lse_merge", "rm_ulysses_permute", "rm_ulysses_permute_qkv",
                  "rm_seq_reorder", "rm_check_device_status", "rm_status_string"):
         assert name in fns
@@ -96,6 +97,33 @@ def test_backward_validation(lib):
     mis = list(base)
     mis[9] = A + 16                                                        # workspace not 256-aligned
     assert lib.rm_ring_attn_bwd(*mis) == 1
+
+
+def test_window_validation(lib):
+    def fwdw(window, S=1024, **kw):
+        return lib.rm_ring_attn_fwd_window(A, A, A, A, A, 1, 4, 2, S, 128, 4, window,
+                                           kw.get("order", 1), kw.get("dtype", 0), 0.088, None)
+    assert fwdw(0) == 1 and fwdw(-3) == 1                      # the window counts keys, >= 1
+    assert fwdw(16, S=0) == 0                                  # empty: nothing to do
+    assert fwdw(16, S=1004) == 1                               # shape rules of the forward
+    assert fwdw(16, order=9) == 1
+    bw = [A] * 10 + [1 << 16, 1, 4, 2, 1024, 128, 4, 64, 1, 0, 0.088, None]
+    assert lib.rm_ring_attn_bwd_window(*bw[:9], None, *bw[10:]) == 1   # no workspace
+    zero = list(bw)
+    zero[17] = 0
+    assert lib.rm_ring_attn_bwd_window(*zero) == 1                     # window 0
+    fp32 = list(bw)
+    fp32[19] = 1
+    assert lib.rm_ring_attn_bwd_window(*fp32) == 2                     # fp32 unsupported
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_window_calls_reach_the_device_without_gpu(lib):
+    # valid arguments pass host validation; with no GPU the CUDA lookup fails
+    assert lib.rm_ring_attn_fwd_window(A, A, A, A, A, 1, 4, 2, 1024, 128, 4, 300, 1, 0, 0.088,
+                                       None) == 3
+    assert lib.rm_ring_attn_fwd_window(A, A, A, A, A, 1, 4, 2, 1024, 64, 4, 5000, 0, 1, 0.125,
+                                       None) == 3
 
 
 def test_layout_validation(lib):
