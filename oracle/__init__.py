@@ -46,14 +46,15 @@ def _L():
         lib.orc_rank_major_position.restype = i64
         lib.orc_rank_major_position.argtypes = [i64, i64, c_int, i64]
         lib.orc_attn_fwd_head.restype = None
-        lib.orc_attn_fwd_head.argtypes = [dp, dp, dp, i64, i64, c_int, i64, c_double, ip, i64, dp, dp]
+        lib.orc_attn_fwd_head.argtypes = [dp, dp, dp, i64, i64, c_int, i64, ip, i64, c_double, ip,
+                                          i64, dp, dp]
         lib.orc_ring_fwd_head.restype = None
-        lib.orc_ring_fwd_head.argtypes = [dp, dp, dp, i64, i64, c_int, i64, c_double, i64, c_int,
-                                          ip, i64, dp, dp]
+        lib.orc_ring_fwd_head.argtypes = [dp, dp, dp, i64, i64, c_int, i64, ip, i64, c_double, i64,
+                                          c_int, ip, i64, dp, dp]
         lib.orc_lse_merge.restype = None
         lib.orc_lse_merge.argtypes = [dp, dp, dp, dp, i64, i64]
         lib.orc_attn_bwd_head.restype = None
-        lib.orc_attn_bwd_head.argtypes = [dp, dp, dp, dp, i64, i64, c_int, i64, c_double,
+        lib.orc_attn_bwd_head.argtypes = [dp, dp, dp, dp, i64, i64, c_int, i64, ip, i64, c_double,
                                           ip, i64, dp, ip, i64, dp, dp]
         lib.orc_ring_owner.restype = i64
         lib.orc_ring_owner.argtypes = [i64, i64, i64]
@@ -163,11 +164,24 @@ def _rows_arg(rows, S):
     return _i64(np.arange(S) if rows is None else rows)
 
 
-def attn_fwd(q, k, v, causal: bool, scale: float = None, rows=None, window: int = 0):
+def _cu_arg(cu_seqlens, S):
+    """Document boundaries as an int64 array (cu[0] = 0, ..., cu[n] = S), or None."""
+    if cu_seqlens is None:
+        return None, 0
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    if cu.ndim != 1 or len(cu) < 2 or cu[0] != 0 or cu[-1] != S or np.any(np.diff(cu) < 0):
+        raise ValueError("cu_seqlens must rise from 0 to S")
+    return cu, len(cu) - 1
+
+
+def attn_fwd(q, k, v, causal: bool, scale: float = None, rows=None, window: int = 0,
+             cu_seqlens=None):
     """Dense softmax attention in natural order.
 
     window: with causal, each query sees its last `window` keys (itself
     included); 0 = no window.
+    cu_seqlens: packed documents [cu[d], cu[d+1]); a query sees keys of its
+    own document only. None = one document.
 
     q [B,H,S,D], k/v [B,Hkv,Sk,D] (numpy or torch, any float dtype; widened to
     fp64 one head at a time); query head h reads KV head h // (H/Hkv).
@@ -179,6 +193,7 @@ def attn_fwd(q, k, v, causal: bool, scale: float = None, rows=None, window: int 
     Hkv, Sk = _shape(k)[1], _shape(k)[2]
     G = H // Hkv
     scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
+    cu, ndoc = _cu_arg(cu_seqlens, Sk)
     r = _rows_arg(rows, S)
     o = np.zeros((B, H, len(r), D))
     lse = np.zeros((B, H, len(r)))
@@ -191,13 +206,14 @@ def attn_fwd(q, k, v, causal: bool, scale: float = None, rows=None, window: int 
                 ob = np.zeros((len(r), D))
                 lb = np.zeros(len(r))
                 lib.orc_attn_fwd_head(_p(qh), _p(kh), _p(vh), Sk, D, int(causal), int(window),
+                                      _p(cu, ctypes.c_int64) if cu is not None else None, ndoc,
                                       scale, _p(r, ctypes.c_int64), len(r), _p(ob), _p(lb))
                 o[b, h], lse[b, h] = ob, lb
     return o, lse
 
 
 def ring_fwd(q, k, v, causal: bool, P: int, order: int, scale: float = None, rows=None,
-             window: int = 0):
+             window: int = 0, cu_seqlens=None):
     """Ring-structured forward: per (rank, step) partials merged step by step.
 
     Same arguments and results as attn_fwd (natural order in and out); the
@@ -207,6 +223,7 @@ def ring_fwd(q, k, v, causal: bool, P: int, order: int, scale: float = None, row
     Hkv = _shape(k)[1]
     G = H // Hkv
     scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
+    cu, ndoc = _cu_arg(cu_seqlens, S)
     r = _rows_arg(rows, S)
     o = np.zeros((B, H, len(r), D))
     lse = np.zeros((B, H, len(r)))
@@ -218,8 +235,10 @@ def ring_fwd(q, k, v, causal: bool, P: int, order: int, scale: float = None, row
                 qh = _f64(_rows_of(q[b, h], r) if rows is not None else q[b, h])
                 ob = np.zeros((len(r), D))
                 lb = np.zeros(len(r))
-                lib.orc_ring_fwd_head(_p(qh), _p(kh), _p(vh), S, D, int(causal), int(window), scale,
-                                      P, order, _p(r, ctypes.c_int64), len(r), _p(ob), _p(lb))
+                lib.orc_ring_fwd_head(_p(qh), _p(kh), _p(vh), S, D, int(causal), int(window),
+                                      _p(cu, ctypes.c_int64) if cu is not None else None, ndoc,
+                                      scale, P, order, _p(r, ctypes.c_int64), len(r), _p(ob),
+                                      _p(lb))
                 o[b, h], lse[b, h] = ob, lb
     return o, lse
 
@@ -237,7 +256,7 @@ def lse_merge(o_acc, lse_acc, o_part, lse_part):
 
 
 def attn_bwd(q, k, v, dout, causal: bool, scale: float = None, qrows=None,
-             krows=None, heads=None, window: int = 0):
+             krows=None, heads=None, window: int = 0, cu_seqlens=None):
     """Gradients of L = sum(dout * O) for dense attention (natural order).
 
     qrows: natural query positions for dQ (None = all); krows: key positions
@@ -250,6 +269,7 @@ def attn_bwd(q, k, v, dout, causal: bool, scale: float = None, qrows=None,
     Hkv = _shape(k)[1]
     G = H // Hkv
     scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
+    cu, ndoc = _cu_arg(cu_seqlens, S)
     qr = _rows_arg(qrows, S)
     kr = _rows_arg(krows, S)
     lib = _L()
@@ -274,6 +294,7 @@ def attn_bwd(q, k, v, dout, causal: bool, scale: float = None, qrows=None,
         dk = np.zeros((max(nk, 1), D))
         dv = np.zeros((max(nk, 1), D))
         lib.orc_attn_bwd_head(_p(qh), _p(kh), _p(vh), _p(doh), S, D, int(causal), int(window),
+                              _p(cu, ctypes.c_int64) if cu is not None else None, ndoc,
                               scale, _p(qr, ctypes.c_int64), nq, _p(dq),
                               _p(kr, ctypes.c_int64), nk, _p(dk), _p(dv))
         if want_q:

@@ -14,6 +14,10 @@
  *     positions ("DeDLOC Guide", Best Practices table, Causal Mask Handling);
  *     with a sliding window of W keys (axolotl-ringmaster README, Status:
  *     sliding-window attention via flash's `window`), also j > i - W;
+ *   - packed variable-length documents (axolotl-ringmaster README, Status:
+ *     packing / varlen): with boundaries cu[0] = 0 <= cu[1] <= ... <= cu[n] = S,
+ *     key j is visible to query i only if both lie in the same document
+ *     [cu[d], cu[d+1]) (and the causal and window rules hold);
  *   - the merge of two partial (O, LSE) pairs by max-shifted exponential weights
  *     ("DeDLOC Guide", section 3 "Online Softmax Rescaling Across Decentralized
  *     Ranks", the alpha/beta equations, in the normalised-output form of Step 3);
@@ -86,17 +90,33 @@ static int rank_holds(int64_t S, int64_t P, int order, int64_t r, int64_t j)
 /* Dense attention of one head, the plain definition.                         */
 /* ------------------------------------------------------------------------- */
 
-/* Visible keys of the query at position i among S keys: [lo, hi).
- * Non-causal: all. Causal: j <= i. Causal with a window of W > 0 keys:
- * i - W < j <= i. */
-static void visible_range(int64_t i, int64_t S, int causal, int64_t window, int64_t* lo,
-                          int64_t* hi)
+/* Which keys a query sees: S tokens, causal flag, window W (0 = none) and the
+ * document boundaries cu[0..ndoc] (cu = NULL: one document of all S tokens). */
+typedef struct {
+    int64_t S;
+    int causal;
+    int64_t window;
+    const int64_t* cu;
+    int64_t ndoc;
+} orc_mask;
+
+/* Visible keys of the query at position i: [lo, hi). The query's document
+ * [cu[d], cu[d+1]) bounds it; causal: j <= i; window of W > 0 keys: j > i - W. */
+static void visible_range(int64_t i, const orc_mask* mk, int64_t* lo, int64_t* hi)
 {
     *lo = 0;
-    *hi = S;
-    if (!causal) return;
-    *hi = i + 1 < S ? i + 1 : S;
-    if (window > 0 && i - window + 1 > 0) *lo = i - window + 1;
+    *hi = mk->S;
+    if (mk->cu) {
+        for (int64_t d = 0; d < mk->ndoc; ++d)
+            if (mk->cu[d] <= i && i < mk->cu[d + 1]) {
+                *lo = mk->cu[d];
+                *hi = mk->cu[d + 1];
+                break;
+            }
+    }
+    if (!mk->causal) return;
+    if (i + 1 < *hi) *hi = i + 1;
+    if (mk->window > 0 && i - mk->window + 1 > *lo) *lo = i - mk->window + 1;
 }
 
 static double dot(const double* a, const double* b, int64_t D)
@@ -107,17 +127,17 @@ static double dot(const double* a, const double* b, int64_t D)
 }
 
 /* For query at natural position i over the visible key set
- * V(i) = {0..S-1} (non-causal), {0..min(i, S-1)} (causal) or, with a window
- * of W > 0 keys, {max(0, i-W+1)..min(i, S-1)}; S keys in k, v:
+ * V(i) = the query's document (non-causal), its part j <= i (causal), and with
+ * a window of W > 0 keys only j > i - W; S keys in k, v:
  *   LSE_i = m + ln sum_j exp(s_ij - m),  m = max_j s_ij
  *   O_i   = sum_j exp(s_ij - LSE_i) v_j
  * scratch must hold S doubles. */
-static void attend_row(const double* qi, const double* k, const double* v, int64_t S,
-                       int64_t D, int causal, int64_t window, double scale, int64_t i,
-                       double* s, double* o, double* lse)
+static void attend_row(const double* qi, const double* k, const double* v, int64_t D,
+                       const orc_mask* mk, double scale, int64_t i, double* s, double* o,
+                       double* lse)
 {
     int64_t j0, n;
-    visible_range(i, S, causal, window, &j0, &n);
+    visible_range(i, mk, &j0, &n);
     double m = -INFINITY;
     for (int64_t j = j0; j < n; ++j) {
         s[j] = scale * dot(qi, k + j * D, D);
@@ -136,19 +156,19 @@ static void attend_row(const double* qi, const double* k, const double* v, int64
 }
 
 /* q holds nrows query rows (row-major [nrows, D]); rows[r] is the natural
- * position of q row r. k, v hold the Sk keys 0..Sk-1. Causal: the query at
- * position i sees keys j <= i. */
+ * position of q row r. k, v hold the Sk keys 0..Sk-1. The mask: causal flag,
+ * window (0 = none), document boundaries cu[0..ndoc] (NULL = one document). */
 void orc_attn_fwd_head(const double* q, const double* k, const double* v, int64_t Sk,
-                       int64_t D, int causal, int64_t window, double scale,
-                       const int64_t* rows, int64_t nrows, double* o, double* lse)
+                       int64_t D, int causal, int64_t window, const int64_t* cu, int64_t ndoc,
+                       double scale, const int64_t* rows, int64_t nrows, double* o, double* lse)
 {
+    const orc_mask mk = {Sk, causal, window, cu, ndoc};
 #pragma omp parallel
     {
         double* s = (double*)malloc(sizeof(double) * (size_t)Sk);
 #pragma omp for schedule(dynamic, 4)
         for (int64_t r = 0; r < nrows; ++r)
-            attend_row(q + r * D, k, v, Sk, D, causal, window, scale, rows[r], s, o + r * D,
-                       lse + r);
+            attend_row(q + r * D, k, v, D, &mk, scale, rows[r], s, o + r * D, lse + r);
         free(s);
     }
 }
@@ -196,9 +216,11 @@ void orc_lse_merge(double* o_acc, double* lse_acc, const double* o_part,
  * order with merge_pair. The result equals the dense definition exactly up to
  * rounding, which the tests check. */
 void orc_ring_fwd_head(const double* q, const double* k, const double* v, int64_t S,
-                       int64_t D, int causal, int64_t window, double scale, int64_t P,
-                       int order, const int64_t* rows, int64_t nrows, double* o, double* lse)
+                       int64_t D, int causal, int64_t window, const int64_t* cu, int64_t ndoc,
+                       double scale, int64_t P, int order, const int64_t* rows, int64_t nrows,
+                       double* o, double* lse)
 {
+    const orc_mask mk = {S, causal, window, cu, ndoc};
 #pragma omp parallel
     {
         double* s = (double*)malloc(sizeof(double) * (size_t)S);
@@ -208,7 +230,7 @@ void orc_ring_fwd_head(const double* q, const double* k, const double* v, int64_
             int64_t x = rows[rr];
             int64_t i = rank_of_position(S, P, order, x);
             int64_t jlo, jhi;
-            visible_range(x, S, causal, window, &jlo, &jhi);
+            visible_range(x, &mk, &jlo, &jhi);
             double* oacc = o + rr * D;
             double lacc = -INFINITY;
             for (int64_t d = 0; d < D; ++d) oacc[d] = 0.0;
@@ -259,9 +281,11 @@ void orc_ring_fwd_head(const double* q, const double* k, const double* v, int64_
  * sum of its query heads' dK/dV, which the caller forms. */
 void orc_attn_bwd_head(const double* q, const double* k, const double* v,
                        const double* dout, int64_t S, int64_t D, int causal, int64_t window,
-                       double scale, const int64_t* qrows, int64_t nq, double* dq,
-                       const int64_t* krows, int64_t nk, double* dk, double* dv)
+                       const int64_t* cu, int64_t ndoc, double scale, const int64_t* qrows,
+                       int64_t nq, double* dq, const int64_t* krows, int64_t nk, double* dk,
+                       double* dv)
 {
+    const orc_mask mk = {S, causal, window, cu, ndoc};
     /* dQ rows: one forward row each, then the sum over its keys. */
 #pragma omp parallel
     {
@@ -271,10 +295,10 @@ void orc_attn_bwd_head(const double* q, const double* k, const double* v,
         for (int64_t r = 0; r < nq; ++r) {
             int64_t i = qrows[r];
             double L;
-            attend_row(q + i * D, k, v, S, D, causal, window, scale, i, s, oi, &L);
+            attend_row(q + i * D, k, v, D, &mk, scale, i, s, oi, &L);
             double delta = dot(dout + i * D, oi, D);
             int64_t j0, n;
-            visible_range(i, S, causal, window, &j0, &n);
+            visible_range(i, &mk, &j0, &n);
             double* g = dq + r * D;
             for (int64_t d = 0; d < D; ++d) g[d] = 0.0;
             for (int64_t j = j0; j < n; ++j) {
@@ -301,7 +325,7 @@ void orc_attn_bwd_head(const double* q, const double* k, const double* v,
         double* oi = (double*)malloc(sizeof(double) * (size_t)D);
 #pragma omp for schedule(dynamic, 16)
         for (int64_t i = i0; i < S; ++i) {
-            attend_row(q + i * D, k, v, S, D, causal, window, scale, i, s, oi, &lse_all[i]);
+            attend_row(q + i * D, k, v, D, &mk, scale, i, s, oi, &lse_all[i]);
             delta_all[i] = dot(dout + i * D, oi, D);
         }
         free(oi);
@@ -313,10 +337,11 @@ void orc_attn_bwd_head(const double* q, const double* k, const double* v,
         double* gk = dk + r * D;
         double* gv = dv + r * D;
         for (int64_t d = 0; d < D; ++d) { gk[d] = 0.0; gv[d] = 0.0; }
-        /* query rows that see key j: i >= j (causal) and i < j + W (window) */
-        int64_t ibeg = causal ? j : 0;
-        int64_t iend = (causal && window > 0 && j + window < S) ? j + window : S;
-        for (int64_t i = ibeg; i < iend; ++i) {
+        /* every query row whose visible range holds key j */
+        for (int64_t i = i0; i < S; ++i) {
+            int64_t lo, hi;
+            visible_range(i, &mk, &lo, &hi);
+            if (j < lo || j >= hi) continue;
             double sij = scale * dot(q + i * D, k + j * D, D);
             double p = exp(sij - lse_all[i]);
             double ds = p * (dot(dout + i * D, v + j * D, D) - delta_all[i]);

@@ -433,3 +433,128 @@ def test_window_backward_finite_differences_and_row_subsets():
                                   heads=([(0, 0)], [(0, 0)]), window=W)
     np.testing.assert_allclose(dq_s[(0, 0)], dq[(0, 0)][rows], atol=1e-13)
     np.testing.assert_allclose(dkv_s[(0, 0)][0], dkv[(0, 0)][0][rows], atol=1e-13)
+
+
+# --- packed variable-length documents (axolotl-ringmaster README, Status:
+# packing / varlen): a query sees keys of its own document [cu[d], cu[d+1])
+# only, with the causal and window rules applied inside it ---
+
+def _doc_ids(cu, S):
+    d = np.zeros(S, dtype=np.int64)
+    for n in range(len(cu) - 1):
+        d[cu[n]:cu[n + 1]] = n
+    return d
+
+
+def _np_doc_attention(q, k, v, cu, causal, W, scale):
+    """Block-diagonal (optionally causal, windowed) attention with numpy/scipy."""
+    B, H, S, D = q.shape
+    G = H // k.shape[1]
+    doc = _doc_ids(cu, S)
+    i = np.arange(S)[:, None]
+    j = np.arange(S)[None, :]
+    hidden = doc[:, None] != doc[None, :]
+    if causal:
+        hidden |= j > i
+        if W:
+            hidden |= j <= i - W
+    o = np.zeros((B, H, S, D))
+    lse = np.zeros((B, H, S))
+    for b in range(B):
+        for h in range(H):
+            s = np.where(hidden, -np.inf, scale * q[b, h] @ k[b, h // G].T)
+            lse[b, h] = logsumexp(s, axis=-1)
+            o[b, h] = np.exp(s - lse[b, h][:, None]) @ v[b, h // G]
+    return o, lse
+
+
+DOCS = [[0, 5, 6, 19, 32], [0, 1, 2, 3, 32], [0, 32], [0, 11, 11, 23, 32]]
+
+
+@pytest.mark.parametrize("cu", DOCS)
+@pytest.mark.parametrize("causal,W", [(True, 0), (False, 0), (True, 4)])
+def test_varlen_forward_matches_numpy_bruteforce(cu, causal, W):
+    S, D = 32, 5
+    q, k, v = _rand((2, 4, S, D), 120), _rand((2, 2, S, D), 121), _rand((2, 2, S, D), 122)
+    o, lse = oracle.attn_fwd(q, k, v, causal, 0.4, window=W, cu_seqlens=cu)
+    o_ref, lse_ref = _np_doc_attention(q, k, v, cu, causal, W, 0.4)
+    np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_varlen_each_document_is_attention_over_itself(causal):
+    # packing must not leak across documents: each document's rows equal the
+    # plain attention of that document taken alone
+    cu = [0, 7, 20, 21, 40]
+    S, D = 40, 6
+    q, k, v = _rand((1, 2, S, D), 130), _rand((1, 1, S, D), 131), _rand((1, 1, S, D), 132)
+    o, lse = oracle.attn_fwd(q, k, v, causal, cu_seqlens=cu)
+    for a, b in zip(cu[:-1], cu[1:]):
+        o_d, lse_d = oracle.attn_fwd(q[:, :, a:b], k[:, :, a:b], v[:, :, a:b], causal)
+        np.testing.assert_allclose(o[:, :, a:b], o_d, rtol=0, atol=1e-14)
+        np.testing.assert_allclose(lse[:, :, a:b], lse_d, rtol=0, atol=1e-14)
+    # a document of one token attends to itself only
+    np.testing.assert_allclose(o[0, :, 20], np.repeat(v[0, :, 20], 2, axis=0), atol=1e-14)
+
+
+def test_varlen_special_cases():
+    S, D = 24, 4
+    q, k, v = _rand((1, 2, S, D), 140), _rand((1, 2, S, D), 141), _rand((1, 2, S, D), 142)
+    for causal in (True, False):
+        # one document is the plain definition; empty documents change nothing
+        a = oracle.attn_fwd(q, k, v, causal, cu_seqlens=[0, S])
+        b = oracle.attn_fwd(q, k, v, causal)
+        np.testing.assert_array_equal(a[0], b[0])
+        c = oracle.attn_fwd(q, k, v, causal, cu_seqlens=[0, 0, 9, 9, 9, S, S])
+        d = oracle.attn_fwd(q, k, v, causal, cu_seqlens=[0, 9, S])
+        np.testing.assert_array_equal(c[0], d[0])
+        # documents of one token: O_i = v_i
+        e, _ = oracle.attn_fwd(q, k, v, causal, cu_seqlens=list(range(S + 1)))
+        np.testing.assert_allclose(e, v, atol=1e-14)
+    with pytest.raises(ValueError):
+        oracle.attn_fwd(q, k, v, True, cu_seqlens=[0, 10, 9, S])
+    with pytest.raises(ValueError):
+        oracle.attn_fwd(q, k, v, True, cu_seqlens=[1, S])
+
+
+@pytest.mark.parametrize("order", [oracle.CONTIGUOUS, oracle.ZIGZAG])
+@pytest.mark.parametrize("P,causal,W", [(2, True, 0), (4, True, 0), (4, False, 0), (3, True, 5)])
+def test_varlen_ring_equals_dense(order, P, causal, W):
+    S, D = 2 * P * 6, 4
+    cu = [0, 5, 17, S - 3, S]
+    q, k, v = _rand((1, 2, S, D), 150 + P), _rand((1, 1, S, D), 151), _rand((1, 1, S, D), 152)
+    o_r, l_r = oracle.ring_fwd(q, k, v, causal, P, order, 0.5, window=W, cu_seqlens=cu)
+    o_d, l_d = _np_doc_attention(q, k, v, cu, causal, W, 0.5)
+    np.testing.assert_allclose(o_r, o_d, atol=1e-13, rtol=0)
+    np.testing.assert_allclose(l_r, l_d, atol=1e-13, rtol=0)
+
+
+@pytest.mark.parametrize("causal,W", [(True, 0), (False, 0), (True, 3)])
+def test_varlen_backward_matches_torch_autograd(causal, W):
+    B, H, Hkv, S, D = 1, 2, 1, 18, 4
+    cu = [0, 4, 5, 13, 18]
+    q, k, v = _rand((B, H, S, D), 160), _rand((B, Hkv, S, D), 161), _rand((B, Hkv, S, D), 162)
+    dout = _rand((B, H, S, D), 163)
+    scale = 0.55
+    tq, tk, tv = (torch.tensor(a, requires_grad=True) for a in (q, k, v))
+    doc = torch.from_numpy(_doc_ids(cu, S))
+    i = torch.arange(S)[:, None]
+    j = torch.arange(S)[None, :]
+    hidden = doc[:, None] != doc[None, :]
+    if causal:
+        hidden = hidden | (j > i)
+        if W:
+            hidden = hidden | (j <= i - W)
+    s = (torch.matmul(tq, tk.repeat_interleave(H // Hkv, 1).transpose(-1, -2)) * scale)
+    s = s.masked_fill(hidden, float("-inf"))
+    o = torch.matmul(torch.softmax(s, -1), tv.repeat_interleave(H // Hkv, 1))
+    (o * torch.tensor(dout)).sum().backward()
+    dq, dkv = oracle.attn_bwd(q, k, v, dout, causal, scale, window=W, cu_seqlens=cu)
+    for h in range(H):
+        np.testing.assert_allclose(dq[(0, h)], tq.grad[0, h].numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(dkv[(0, 0)][0], tk.grad[0, 0].numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(dkv[(0, 0)][1], tv.grad[0, 0].numpy(), atol=1e-12, rtol=0)
+    # per document, sum_j dK_j = 0 (softmax shift invariance inside each document)
+    for a, b in zip(cu[:-1], cu[1:]):
+        assert np.abs(dkv[(0, 0)][0][a:b].sum(0)).max() < 1e-12
