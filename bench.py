@@ -43,7 +43,8 @@ def parse_args():
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--only", choices=["all", "fwd", "permute", "bwd", "window"], default="all",
+    p.add_argument("--only", choices=["all", "fwd", "permute", "bwd", "window", "packed"],
+                   default="all",
                    help="restrict to one kernel (used for profiling runs)")
     p.add_argument("--skip-cpu", action="store_true", help="skip the CPU oracle baseline")
     p.add_argument("--skip-e2e", action="store_true")
@@ -342,12 +343,15 @@ def bench_permute(args, dev, stream):
             "gbs": moved / ms / 1e6, "launches": steps + max(3, args.warmup)}
 
 
-def bench_window(args, dev, stream):
-    """Sliding-window forward: the 32k GQA layer with a 4096-key causal window."""
+def bench_masked(args, dev, stream, name):
+    """Forward with a sparser mask: the 32k GQA layer with a 4096-key causal
+    window, or over packed documents."""
     import torch
     import ring_ulysses_sequence_b200 as rm
     from ring_ulysses_sequence_b200.synth import WORKLOADS
-    w = WORKLOADS["ring_fwd_bf16_S32k_gqa_causal_zigzag_window4k"]
+    w = WORKLOADS[name]
+    table = rm.varlen_bounds(list(w.cu_seqlens), w.S, w.causal, device=dev) if w.cu_seqlens \
+        else None
     g = torch.Generator(device=dev)
     g.manual_seed(w.seed)
     q, k, v = ((torch.randn(s, generator=g, device=dev) * w.input_scale).to(w.dtype)
@@ -356,8 +360,8 @@ def bench_window(args, dev, stream):
     lse = torch.empty((w.B, w.H, w.S), dtype=torch.float32, device=dev)
 
     def step():
-        rm.ring_attn_fwd(q, k, v, w.P, True, w.order, out=o, lse=lse, stream=stream,
-                         window=w.window)
+        rm.ring_attn_fwd(q, k, v, w.P, w.causal, w.order, out=o, lse=lse, stream=stream,
+                         window=w.window, bounds=table)
 
     with torch.cuda.stream(stream):
         for _ in range(max(3, args.warmup)):
@@ -367,7 +371,8 @@ def bench_window(args, dev, stream):
     ms = time_on_stream(step, steps, stream) / steps
     if rm.native.rm_check_device_status(stream) != 0:
         raise RuntimeError("device watchdog fired during the window benchmark")
-    return {"workload": w.name, "window": w.window, "ms_per_launch": ms,
+    return {"workload": w.name, "window": w.window, "docs": max(len(w.cu_seqlens) - 1, 0),
+            "ms_per_launch": ms,
             "tflops": w.fwd_flops() / ms / 1e9, "flops_per_launch": w.fwd_flops(),
             "launches": steps + max(3, args.warmup)}
 
@@ -427,7 +432,11 @@ def main():
         if rank == 0 and args.only in ("all", "permute"):
             out["permute"] = bench_permute(args, dev, stream)
         if rank == 0 and args.only in ("all", "window"):
-            out["window"] = bench_window(args, dev, stream)
+            out["window"] = bench_masked(args, dev, stream,
+                                         "ring_fwd_bf16_S32k_gqa_causal_zigzag_window4k")
+        if rank == 0 and args.only in ("all", "packed"):
+            out["packed"] = bench_masked(args, dev, stream,
+                                         "ring_fwd_bf16_S32k_gqa_causal_zigzag_packed")
         if rank == 0 and args.only in ("all", "bwd"):
             try:
                 out["bwd"] = bench_backward(args, dev, stream)
@@ -486,11 +495,13 @@ def main():
                          "unit": "GB/s", "frac": p["gbs"] / peaks["hbm_gbs"],
                          "peak_source": f"{peak_src} hbm_gbs",
                          "bytes_per_launch": p["bytes_per_launch"]}}
-    if "window" in out:
-        x = out["window"]
-        extra["ring_attn_fwd_window"] = {
-            "workload": x["workload"], "window": x["window"], "ms": x["ms_per_launch"],
-            "TFLOPS": x["tflops"],
+    for key, label in (("window", "ring_attn_fwd_window"), ("packed", "ring_attn_fwd_varlen")):
+        if key not in out:
+            continue
+        x = out[key]
+        extra[label] = {
+            "workload": x["workload"], "window": x["window"], "docs": x["docs"],
+            "ms": x["ms_per_launch"], "TFLOPS": x["tflops"],
             "roofline": {"bound": "tensor", "achieved": x["tflops"], "peak": peaks["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": x["tflops"] / peaks["bf16_tflops"],
                          "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)",

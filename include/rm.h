@@ -120,6 +120,50 @@ RM_API rm_status rm_ring_attn_fwd_window(const void* q, const void* k, const voi
                                          cudaStream_t stream);
 
 /*
+ * rm_varlen_bounds_size / rm_varlen_bounds — the per-token visibility table of
+ * packed variable-length documents (axolotl-ringmaster README, Status table:
+ * packing / varlen).
+ *
+ * The S tokens (natural order) are the concatenation of n_docs documents with
+ * boundaries cu_seqlens[0] = 0 <= cu_seqlens[1] <= ... <= cu_seqlens[n_docs] =
+ * S (empty documents allowed). A query sees only keys of its own document,
+ * and within it keys j <= i when causal, and j > i - window when window > 0
+ * (causal only; window >= S means none). The ring layout (contiguous or
+ * zigzag) shards the packed sequence as one sequence; masks use global
+ * positions, so results do not depend on P or the order.
+ *
+ *   cu_seqlens : HOST int32 array of n_docs + 1 boundaries, checked on the host
+ *                (RM_ERR_INVALID_ARG if it does not rise from 0 to S)
+ *   bounds     : device buffer of at least rm_varlen_bounds_size(S, n_docs)
+ *                bytes, 256-byte aligned, owned by the caller. It receives one
+ *                int4 per token {lo, hi, imin, imax}: query i sees keys
+ *                lo..hi, key j is seen by queries imin..imax (natural
+ *                positions), followed by a copy of cu_seqlens.
+ * The host array may be reused as soon as the call returns. Build the table
+ * once per batch layout and pass it to every rm_ring_attn_*_varlen call with
+ * the same S (each batch row uses the same documents).
+ */
+RM_API size_t rm_varlen_bounds_size(int S, int n_docs);
+
+RM_API rm_status rm_varlen_bounds(const int* cu_seqlens, int n_docs, int S, int causal,
+                                  int window, void* bounds, size_t bounds_bytes,
+                                  cudaStream_t stream);
+
+/*
+ * rm_ring_attn_fwd_varlen — rm_ring_attn_fwd over packed documents.
+ *
+ * Arguments, layouts and shape rules as rm_ring_attn_fwd; the mask (causal or
+ * not, window, documents) comes from `bounds`, a table made by
+ * rm_varlen_bounds for this S. Key tiles no query row can see (other
+ * documents, before a window) are skipped, so the work follows the documents'
+ * lengths.
+ */
+RM_API rm_status rm_ring_attn_fwd_varlen(const void* q, const void* k, const void* v, void* o,
+                                         float* lse, const void* bounds, int B, int H, int Hkv,
+                                         int S, int D, int P, rm_order order, rm_dtype dtype,
+                                         float scale, cudaStream_t stream);
+
+/*
  * rm_ring_attn_bwd — gradients of L = sum(dO * O) through the ring forward
  * (axolotl-ringmaster README: flash-style reverse-ring backward; gradients
  * accumulate in fp32 across ring steps).
@@ -159,6 +203,19 @@ RM_API rm_status rm_ring_attn_bwd_window(const void* q, const void* k, const voi
                                          float* dq, float* dk, float* dv, void* workspace,
                                          size_t workspace_bytes, int B, int H, int Hkv, int S,
                                          int D, int P, int window, rm_order order,
+                                         rm_dtype dtype, float scale, cudaStream_t stream);
+
+/*
+ * rm_ring_attn_bwd_varlen — rm_ring_attn_bwd through rm_ring_attn_fwd_varlen:
+ * the same gradients with P_ij = 0 for pairs the documents' mask hides.
+ * Arguments, layouts, workspace, outputs and status codes as rm_ring_attn_bwd;
+ * `bounds` as for the forward (the same table the forward used).
+ */
+RM_API rm_status rm_ring_attn_bwd_varlen(const void* q, const void* k, const void* v,
+                                         const void* o, const float* lse, const void* dout,
+                                         float* dq, float* dk, float* dv, const void* bounds,
+                                         void* workspace, size_t workspace_bytes, int B, int H,
+                                         int Hkv, int S, int D, int P, rm_order order,
                                          rm_dtype dtype, float scale, cudaStream_t stream);
 
 /*

@@ -16,7 +16,7 @@ from .native import (RM_DTYPE_BF16, RM_DTYPE_FP32, RM_HEAD_TO_SEQ,
                      RM_NATURAL_TO_RANK_MAJOR, RM_ORDER_CONTIGUOUS, RM_ORDER_ZIGZAG,
                      RM_RANK_MAJOR_TO_NATURAL, RM_SEQ_TO_HEAD, RMError)
 
-__all__ = ["ring_attn_fwd", "ring_attn_bwd", "lse_merge_", "ulysses_permute",
+__all__ = ["ring_attn_fwd", "ring_attn_bwd", "varlen_bounds", "lse_merge_", "ulysses_permute",
            "ulysses_permute_qkv", "seq_reorder", "native", "RMError"]
 
 _ORDERS = {"contiguous": RM_ORDER_CONTIGUOUS, "zigzag": RM_ORDER_ZIGZAG}
@@ -40,11 +40,25 @@ def _need(t, name):
         raise ValueError(f"{name} must be a contiguous CUDA tensor")
 
 
+def varlen_bounds(cu_seqlens, S, causal=True, window=0, device=None, stream=None):
+    """Visibility table of packed documents (boundaries cu_seqlens, natural
+    positions, from 0 to S) for the *_varlen calls: a uint8 device tensor."""
+    import torch
+    n_docs = len(cu_seqlens) - 1
+    nbytes = native.rm_varlen_bounds_size(S, n_docs)
+    table = torch.empty(max(nbytes, 256), dtype=torch.uint8,
+                        device=device if device is not None else "cuda")
+    native.rm_varlen_bounds(cu_seqlens, n_docs, S, causal, window, table, table.numel(), stream)
+    return table
+
+
 def ring_attn_fwd(q, k, v, P, causal=True, order="zigzag", scale=None, out=None, lse=None,
-                  stream=None, window=0):
+                  stream=None, window=0, bounds=None):
     """Ring attention forward. q [B,H,S,D], k/v [B,Hkv,S,D] (rank-major S).
 
     window > 0 (causal only): query i sees keys i - window < j <= i.
+    bounds: a varlen_bounds() table (packed documents); it carries the mask,
+    and causal/window are then ignored.
     Returns (O [B,H,S,D] in q's dtype, LSE [B,H,S] float32).
     """
     import torch
@@ -57,7 +71,10 @@ def ring_attn_fwd(q, k, v, P, causal=True, order="zigzag", scale=None, out=None,
     if lse is None:
         lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
-    if window:
+    if bounds is not None:
+        native.rm_ring_attn_fwd_varlen(q, k, v, out, lse, bounds, B, H, Hkv, S, D, P,
+                                       _order(order), _dtype_code(q), scale, stream)
+    elif window:
         if not causal:
             raise ValueError("a sliding window needs causal=True")
         native.rm_ring_attn_fwd_window(q, k, v, out, lse, B, H, Hkv, S, D, P, window,
@@ -69,10 +86,10 @@ def ring_attn_fwd(q, k, v, P, causal=True, order="zigzag", scale=None, out=None,
 
 
 def ring_attn_bwd(q, k, v, o, lse, dout, P, causal=True, order="zigzag", scale=None,
-                  workspace=None, stream=None, window=0):
+                  workspace=None, stream=None, window=0, bounds=None):
     """Ring attention backward. Returns fp32 (dQ, dK, dV).
 
-    window: as in ring_attn_fwd (o and lse must come from that window).
+    window, bounds: as in ring_attn_fwd (o and lse must come from that mask).
     """
     import torch
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (lse, "lse"), (dout, "dout")):
@@ -86,7 +103,11 @@ def ring_attn_bwd(q, k, v, o, lse, dout, P, causal=True, order="zigzag", scale=N
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
-    if window:
+    if bounds is not None:
+        native.rm_ring_attn_bwd_varlen(q, k, v, o, lse, dout, dq, dk, dv, bounds, workspace,
+                                       workspace.numel(), B, H, Hkv, S, D, P, _order(order),
+                                       _dtype_code(q), scale, stream)
+    elif window:
         if not causal:
             raise ValueError("a sliding window needs causal=True")
         native.rm_ring_attn_bwd_window(q, k, v, o, lse, dout, dq, dk, dv, workspace,

@@ -116,7 +116,8 @@ static rm_status window_arg(int window, int S, int* out) {
 
 static rm_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse,
                           int B, int H, int Hkv, int S, int D, int P, int causal, int window,
-                          rm_order order, rm_dtype dtype, float scale, cudaStream_t stream) {
+                          const void* bounds, rm_order order, rm_dtype dtype, float scale,
+                          cudaStream_t stream) {
     const int tile_q = dtype == RM_DTYPE_BF16 ? 128 : 64;
     rm_status st = check_attn(q, k, v, B, H, Hkv, S, D, P, order, dtype, scale, tile_q);
     if (st != RM_OK) return st;
@@ -125,7 +126,7 @@ static rm_status fwd_impl(const void* q, const void* k, const void* v, void* o, 
     LaunchCtx ctx;
     if ((st = get_ctx(stream, &ctx)) != RM_OK) return st;
     AttnShape sh{B, H, Hkv, S, D, P, causal ? 1 : 0, order == RM_ORDER_ZIGZAG ? 1 : 0, scale,
-                 window};
+                 window, bounds};
     cudaError_t e = dtype == RM_DTYPE_BF16
                         ? launch_fwd_tc(sh, q, k, v, o, lse, ctx)
                         : launch_fwd_fp32(sh, static_cast<const float*>(q),
@@ -138,8 +139,13 @@ static rm_status fwd_impl(const void* q, const void* k, const void* v, void* o, 
 static rm_status bwd_impl(const void* q, const void* k, const void* v, const void* o,
                           const float* lse, const void* dout, float* dq, float* dk, float* dv,
                           void* workspace, size_t workspace_bytes, int B, int H, int Hkv, int S,
-                          int D, int P, int causal, int window, rm_order order, rm_dtype dtype,
-                          float scale, cudaStream_t stream);
+                          int D, int P, int causal, int window, const void* bounds,
+                          rm_order order, rm_dtype dtype, float scale, cudaStream_t stream);
+
+// Layout of a varlen bounds buffer: S int4 entries, then (256-byte aligned) a
+// device copy of the n_docs + 1 boundaries the entries were built from.
+static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+static size_t varlen_table_bytes(int S) { return align256(static_cast<size_t>(S) * 16); }
 
 }  // namespace rm
 
@@ -192,7 +198,8 @@ rm_status rm_watchdog_selftest(uint64_t timeout_ns, cudaStream_t stream) {
 rm_status rm_ring_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                            int B, int H, int Hkv, int S, int D, int P, int causal,
                            rm_order order, rm_dtype dtype, float scale, cudaStream_t stream) {
-    return fwd_impl(q, k, v, o, lse, B, H, Hkv, S, D, P, causal, 0, order, dtype, scale, stream);
+    return fwd_impl(q, k, v, o, lse, B, H, Hkv, S, D, P, causal, 0, nullptr, order, dtype, scale,
+                    stream);
 }
 
 rm_status rm_ring_attn_fwd_window(const void* q, const void* k, const void* v, void* o,
@@ -202,7 +209,45 @@ rm_status rm_ring_attn_fwd_window(const void* q, const void* k, const void* v, v
     int w = 0;
     rm_status st = window_arg(window, S, &w);
     if (st != RM_OK) return st;
-    return fwd_impl(q, k, v, o, lse, B, H, Hkv, S, D, P, 1, w, order, dtype, scale, stream);
+    return fwd_impl(q, k, v, o, lse, B, H, Hkv, S, D, P, 1, w, nullptr, order, dtype, scale, stream);
+}
+
+size_t rm_varlen_bounds_size(int S, int n_docs) {
+    if (S <= 0 || n_docs <= 0) return 0;
+    return varlen_table_bytes(S) + align256(static_cast<size_t>(n_docs + 1) * 4);
+}
+
+rm_status rm_varlen_bounds(const int* cu_seqlens, int n_docs, int S, int causal, int window,
+                           void* bounds, size_t bounds_bytes, cudaStream_t stream) {
+    if (n_docs <= 0 || S < 0 || window < 0 || !cu_seqlens) return RM_ERR_INVALID_ARG;
+    if (window > 0 && !causal) return RM_ERR_INVALID_ARG;
+    if (cu_seqlens[0] != 0 || cu_seqlens[n_docs] != S) return RM_ERR_INVALID_ARG;
+    for (int d = 0; d < n_docs; ++d)
+        if (cu_seqlens[d] > cu_seqlens[d + 1]) return RM_ERR_INVALID_ARG;
+    if (S == 0) return RM_OK;
+    if (!bounds || (reinterpret_cast<uintptr_t>(bounds) & 255u) != 0) return RM_ERR_INVALID_ARG;
+    if (bounds_bytes < rm_varlen_bounds_size(S, n_docs)) return RM_ERR_INVALID_ARG;
+    if (window >= S) window = 0;
+    LaunchCtx ctx;
+    rm_status st = get_ctx(stream, &ctx);
+    if (st != RM_OK) return st;
+    int* cu_dev = reinterpret_cast<int*>(static_cast<char*>(bounds) + varlen_table_bytes(S));
+    // from pageable host memory: the host array may be reused once this returns
+    cudaError_t e = cudaMemcpyAsync(cu_dev, cu_seqlens, static_cast<size_t>(n_docs + 1) * 4,
+                                    cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = launch_varlen_bounds(cu_dev, n_docs, S, causal ? 1 : 0, window, bounds, ctx);
+    return e == cudaSuccess ? RM_OK : cuda_fail(e);
+}
+
+rm_status rm_ring_attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                                  const void* bounds, int B, int H, int Hkv, int S, int D, int P,
+                                  rm_order order, rm_dtype dtype, float scale,
+                                  cudaStream_t stream) {
+    if (S > 0 && B > 0 && (!bounds || (reinterpret_cast<uintptr_t>(bounds) & 255u) != 0))
+        return RM_ERR_INVALID_ARG;
+    return fwd_impl(q, k, v, o, lse, B, H, Hkv, S, D, P, 1, 0, bounds, order, dtype, scale,
+                    stream);
 }
 
 size_t rm_ring_attn_bwd_workspace_size(int B, int H, int S) {
@@ -217,7 +262,7 @@ rm_status rm_ring_attn_bwd(const void* q, const void* k, const void* v, const vo
                            int S, int D, int P, int causal, rm_order order, rm_dtype dtype,
                            float scale, cudaStream_t stream) {
     return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv, S, D,
-                    P, causal, 0, order, dtype, scale, stream);
+                    P, causal, 0, nullptr, order, dtype, scale, stream);
 }
 
 rm_status rm_ring_attn_bwd_window(const void* q, const void* k, const void* v, const void* o,
@@ -229,7 +274,19 @@ rm_status rm_ring_attn_bwd_window(const void* q, const void* k, const void* v, c
     rm_status st = window_arg(window, S, &w);
     if (st != RM_OK) return st;
     return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv, S, D,
-                    P, 1, w, order, dtype, scale, stream);
+                    P, 1, w, nullptr, order, dtype, scale, stream);
+}
+
+rm_status rm_ring_attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                                  const float* lse, const void* dout, float* dq, float* dk,
+                                  float* dv, const void* bounds, void* workspace,
+                                  size_t workspace_bytes, int B, int H, int Hkv, int S, int D,
+                                  int P, rm_order order, rm_dtype dtype, float scale,
+                                  cudaStream_t stream) {
+    if (S > 0 && B > 0 && (!bounds || (reinterpret_cast<uintptr_t>(bounds) & 255u) != 0))
+        return RM_ERR_INVALID_ARG;
+    return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv, S, D,
+                    P, 1, 0, bounds, order, dtype, scale, stream);
 }
 
 }  // extern "C"
@@ -239,8 +296,8 @@ namespace rm {
 static rm_status bwd_impl(const void* q, const void* k, const void* v, const void* o,
                           const float* lse, const void* dout, float* dq, float* dk, float* dv,
                           void* workspace, size_t workspace_bytes, int B, int H, int Hkv, int S,
-                          int D, int P, int causal, int window, rm_order order, rm_dtype dtype,
-                          float scale, cudaStream_t stream) {
+                          int D, int P, int causal, int window, const void* bounds,
+                          rm_order order, rm_dtype dtype, float scale, cudaStream_t stream) {
     rm_status st = check_attn(q, k, v, B, H, Hkv, S, D, P, order, dtype, scale, 128);
     if (st != RM_OK) return st;
     if (dtype != RM_DTYPE_BF16) return RM_ERR_UNSUPPORTED;
@@ -253,7 +310,7 @@ static rm_status bwd_impl(const void* q, const void* k, const void* v, const voi
     LaunchCtx ctx;
     if ((st = get_ctx(stream, &ctx)) != RM_OK) return st;
     AttnShape sh{B, H, Hkv, S, D, P, causal ? 1 : 0, order == RM_ORDER_ZIGZAG ? 1 : 0, scale,
-                 window};
+                 window, bounds};
     cudaError_t e = launch_bwd(sh, q, k, v, o, lse, dout, dq, dk, dv,
                                static_cast<float*>(workspace), ctx);
     return e == cudaSuccess ? RM_OK : cuda_fail(e);

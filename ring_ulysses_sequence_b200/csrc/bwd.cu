@@ -70,8 +70,7 @@ struct BwdArgs {
     unsigned* status;
     unsigned long long timeout_ns;
     int B, H, Hkv, S, P, causal, G, n_items;
-    int window;      // causal left window in keys; 0 = none
-    unsigned band;   // window, or 2^31 - 1 without one: the visible width of a row
+    MaskSpec mk;     // which keys each query sees
     float scale, scale_log2;
     RingLayout lay;
 };
@@ -106,21 +105,26 @@ __device__ __forceinline__ KvItem decode_kv_item(const BwdArgs& a, int w) {
 
 // Query tiles (head, slot, class) that see a key tile, in reverse-ring order:
 // step t visits rank (r + t) mod P; heads of the group innermost. A rank's
-// block is one (contiguous) or two (zigzag) runs of consecutive positions, and
-// the query tiles that see a causal key tile form a suffix of each run (with a
-// window, an interval of it): O(1) work per returned tile, no division. qpos
-// holds the natural position of the query tile last returned.
+// block is one (contiguous) or two (zigzag) runs of consecutive positions. The
+// queries that see any key of the tile form one interval [imin(first key),
+// imax(last key)] (the bounds are monotone), so the query tiles to visit in a
+// run are an interval too: O(1) work per returned tile, no division. qpos holds
+// the natural position of the query tile last returned.
 struct QIter {
-    const BwdArgs* a;
     int rank, kpos, g, t, run, u, u_end, s0, p0, hh, cls, qslot, qpos;
-    __device__ __forceinline__ QIter(const BwdArgs& args, const KvItem& it)
-        : a(&args), rank(it.rank), kpos(it.kpos), g(it.g), t(0), run(-1), u(0), u_end(0), s0(0),
-          p0(0), hh(args.G), cls(kSkip), qslot(0), qpos(0) {}
-    __device__ __forceinline__ bool next(int& h, int& slot, int& c) {
-        const RingLayout& lay = a->lay;
+    int2 cf, cl;  // {imin, imax} of the key tile's first and last key
+    __device__ __forceinline__ QIter(const BwdArgs& a, const KvItem& it)
+        : rank(it.rank), kpos(it.kpos), g(it.g), t(0), run(-1), u(0), u_end(0), s0(0), p0(0),
+          hh(a.G), cls(kSkip), qslot(0), qpos(0) {
+        cf = col_bounds(a.mk, it.kpos);
+        cl = col_bounds(a.mk, it.kpos + kT - 1);
+    }
+    // `a` is the kernel's parameter block itself
+    __device__ __forceinline__ bool next(const BwdArgs& a, int& h, int& slot, int& c) {
+        const RingLayout& lay = a.lay;
         for (;;) {
-            if (hh < a->G) {
-                h = g * a->G + hh++;
+            if (hh < a.G) {
+                h = g * a.G + hh++;
                 slot = qslot;
                 c = cls;
                 return true;
@@ -136,16 +140,13 @@ struct QIter {
                 const int ctiles = (lay.zigzag ? lay.c : lay.L) / kT;
                 s0 = i * lay.L + run * lay.c;
                 p0 = lay.zigzag ? (run == 0 ? i * lay.c : (2 * lay.P - 1 - i) * lay.c) : i * lay.L;
-                u_end = ctiles;
-                u = a->causal ? min(ctiles, max((kpos - p0) >> 7, 0)) : 0;  // first tile at or after the key
-                // window: the last query tile whose first row still sees the
-                // key tile's last key, qp <= kpos + 127 + W - 1
-                if (a->causal && a->window)
-                    u_end = min(ctiles, max(((kpos + a->window + (kT - 2) - p0) >> 7) + 1, 0));
+                // query tiles meeting [cf.x, cl.y]
+                u = max(0, ceil_div128(cf.x - (kT - 1) - p0));
+                u_end = min(ctiles, max(((cl.y - p0) >> 7) + 1, 0));
             }
             qslot = s0 + u * kT;
             qpos = p0 + u * kT;
-            cls = band_tile_class(a->causal, a->window, qpos - kpos);
+            cls = class_from_cols(cf, cl, qpos);
             ++u;
             hh = 0;
         }
@@ -245,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
                 }
                 QIter qi(a, it);
                 int h, qslot, cls;
-                while (ok && qi.next(h, qslot, cls)) {
+                while (ok && qi.next(a, h, qslot, cls)) {
                     const int st = fills % kStages;
                     const uint32_t use = fills / kStages;
                     if (use > 0) ok = mbar_wait(smem_u32(&bars.st_empty[st]), (use - 1) & 1, wd);
@@ -283,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
                 ok = mbar_wait(smem_u32(&bars.res_full), items & 1, wd);
                 if (!ok) break;
                 tc_fence_after();
-                for (int j = 0; ok && qi.next(qh, qs, qc); ++j) {
+                for (int j = 0; ok && qi.next(a, qh, qs, qc); ++j) {
                     const int st = uses % kStages;
                     ok = mbar_wait(smem_u32(&bars.st_full[st]), (uses / kStages) & 1, wd);
                     if (!ok) break;
@@ -327,11 +328,17 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
             const KvItem it = decode_kv_item(a, w);
             QIter qi(a, it);
             int h, qslot, cls;
-            while (ok && qi.next(h, qslot, cls)) {
+            while (ok && qi.next(a, h, qslot, cls)) {
                 const int st = uses % kStages;
                 ++uses;
-                // key row r sees query column c iff 0 <= c - lo < band
-                const int lo = r - (qi.qpos - it.kpos);
+                // key row r sees query column c iff imin(j) <= qpos + c <= imax(j)
+                int lo = 0;
+                unsigned wq = 0;
+                if (cls == kMask) {
+                    const int2 cb = col_bounds(a.mk, it.kpos + r);
+                    lo = cb.x - qi.qpos;
+                    wq = static_cast<unsigned>(cb.y - cb.x);
+                }
                 const float* lse_s = reinterpret_cast<const float*>(
                     smem + 2 * BCfg<D>::kTile + st * BCfg<D>::kStageKV + 2 * BCfg<D>::kTile);
                 const float* del_s = lse_s + kT;
@@ -364,8 +371,8 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
                             float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
                             if (cls == kMask) {
                                 const int q0 = 64 * wg + 32 * qq + c;
-                                if (static_cast<unsigned>(q0 - lo) >= a.band) p0 = 0.f;
-                                if (static_cast<unsigned>(q0 + 1 - lo) >= a.band) p1 = 0.f;
+                                if (static_cast<unsigned>(q0 - lo) > wq) p0 = 0.f;
+                                if (static_cast<unsigned>(q0 + 1 - lo) > wq) p1 = 0.f;
                             }
                             const uint64_t pp = pk2(p0, p1);
                             const uint64_t dd = mul2(pp, sub2(pk2(__uint_as_float(dpv[c]), __uint_as_float(dpv[c + 1])),
@@ -421,18 +428,20 @@ __device__ __forceinline__ QItem decode_q_item(const BwdArgs& a, int w) {
     return it;
 }
 
-// Key tiles a query tile sees, in ring order: step t visits owner (i - t) mod P;
-// within each run of an owner's block the visible tiles are a prefix (with a
-// window, an interval). kpos holds the natural position of the tile last
-// returned.
+// Key tiles a query tile sees, in ring order: step t visits owner (i - t) mod P.
+// The keys the tile's rows see form one interval [lo(first row), hi(last
+// row)], so within each run of an owner's block the tiles to visit are an
+// interval. kpos holds the natural position of the tile last returned.
 struct KIter {
-    const BwdArgs* a;
     int rank, qpos, t, run, u, u_end, s0, p0, kpos;
-    __device__ __forceinline__ KIter(const BwdArgs& args, const QItem& it)
-        : a(&args), rank(it.rank), qpos(it.pos), t(0), run(-1), u(0), u_end(0), s0(0), p0(0),
-          kpos(0) {}
-    __device__ __forceinline__ bool next(int& kslot, int& cls) {
-        const RingLayout& lay = a->lay;
+    int2 rf, rl;  // {lo, hi} of the query tile's first and last row
+    __device__ __forceinline__ KIter(const BwdArgs& a, const QItem& it)
+        : rank(it.rank), qpos(it.pos), t(0), run(-1), u(0), u_end(0), s0(0), p0(0), kpos(0) {
+        rf = row_bounds(a.mk, it.pos);
+        rl = row_bounds(a.mk, it.pos + kT - 1);
+    }
+    __device__ __forceinline__ bool next(const BwdArgs& a, int& kslot, int& cls) {
+        const RingLayout& lay = a.lay;
         while (u >= u_end) {
             const int runs = lay.zigzag ? 2 : 1;
             if (++run == runs) {
@@ -443,14 +452,13 @@ struct KIter {
             const int ctiles = (lay.zigzag ? lay.c : lay.L) / kT;
             s0 = r * lay.L + run * lay.c;
             p0 = lay.zigzag ? (run == 0 ? r * lay.c : (2 * lay.P - 1 - r) * lay.c) : r * lay.L;
-            u = 0;
-            u_end = a->causal ? min(ctiles, max(((qpos - p0) >> 7) + 1, 0)) : ctiles;
-            // window: the first tile whose last key is inside row 0's window
-            if (a->causal && a->window) u = max(0, ceil_div128(qpos - a->window - (kT - 2) - p0));
+            // key tiles meeting [rf.x, rl.y]
+            u = max(0, ceil_div128(rf.x - (kT - 1) - p0));
+            u_end = min(ctiles, max(((rl.y - p0) >> 7) + 1, 0));
         }
         kslot = s0 + u * kT;
         kpos = p0 + u * kT;
-        cls = band_tile_class(a->causal, a->window, qpos - kpos);
+        cls = class_from_rows(rf, rl, kpos);
         ++u;
         return true;
     }
@@ -511,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
                 }
                 KIter ki(a, it);
                 int kslot, cls;
-                while (ok && ki.next(kslot, cls)) {
+                while (ok && ki.next(a, kslot, cls)) {
                     const int st = fills % kStages;
                     const uint32_t use = fills / kStages;
                     if (use > 0) ok = mbar_wait(smem_u32(&bars.st_empty[st]), (use - 1) & 1, wd);
@@ -547,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
                 ok = mbar_wait(smem_u32(&bars.res_full), items & 1, wd);
                 if (!ok) break;
                 tc_fence_after();
-                for (int j = 0; ok && ki.next(ks, kc); ++j) {
+                for (int j = 0; ok && ki.next(a, ks, kc); ++j) {
                     const int st = uses % kStages;
                     ok = mbar_wait(smem_u32(&bars.st_full[st]), (uses / kStages) & 1, wd);
                     if (!ok) break;
@@ -592,9 +600,15 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
             const float delta = a.delta[qrow];
             KIter ki(a, it);
             int kslot, cls;
-            while (ok && ki.next(kslot, cls)) {
-                // query row r sees key column c iff 0 <= hi - c < band
-                const int hi = r + it.pos - ki.kpos;
+            while (ok && ki.next(a, kslot, cls)) {
+                // query row r sees key column c iff lo(i) <= kpos + c <= hi(i)
+                int lo = 0;
+                unsigned wk = 0;
+                if (cls == kMask) {
+                    const int2 rb = row_bounds(a.mk, it.pos + r);
+                    lo = rb.x - ki.kpos;
+                    wk = static_cast<unsigned>(rb.y - rb.x);
+                }
                 ok = mbar_wait(smem_u32(&bars.s_full), (s_cnt++) & 1, wd);
                 if (!ok) break;
                 tc_fence_after();
@@ -610,8 +624,8 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
                     upk2(fma2(pk2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, nlse2), x0, x1);
                     float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
                     if (cls == kMask) {
-                        if (static_cast<unsigned>(hi - k0) >= a.band) p0 = 0.f;
-                        if (static_cast<unsigned>(hi - k0 - 1) >= a.band) p1 = 0.f;
+                        if (static_cast<unsigned>(k0 - lo) > wk) p0 = 0.f;
+                        if (static_cast<unsigned>(k0 + 1 - lo) > wk) p1 = 0.f;
                     }
                     float d0, d1;
                     upk2(mul2(pk2(p0, p1), sub2(pk2(__uint_as_float(dpv[c]), __uint_as_float(dpv[c + 1])), del2)), d0, d1);
@@ -727,8 +741,7 @@ cudaError_t launch_bwd(const AttnShape& sh, const void* q, const void* k, const 
     a.P = sh.P;
     a.causal = sh.causal;
     a.G = sh.H / sh.Hkv;
-    a.window = sh.causal ? sh.window : 0;
-    a.band = a.window ? static_cast<unsigned>(a.window) : 0x7fffffffu;
+    a.mk = MaskSpec{static_cast<const int4*>(sh.bounds), sh.S, sh.causal, sh.causal ? sh.window : 0};
     a.scale = sh.scale;
     a.scale_log2 = sh.scale * kLog2e;
     a.lay = RingLayout{sh.S, sh.P, sh.S / sh.P, sh.zigzag ? sh.S / (2 * sh.P) : sh.S / sh.P, sh.zigzag};

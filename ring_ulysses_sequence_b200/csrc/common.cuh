@@ -39,19 +39,52 @@ struct RingLayout {
     }
 };
 
-// Class of a (128-query tile, 128-key tile) pair from d = qpos - kpos, the
-// difference of the tiles' first natural positions (a multiple of 128). The
-// mask is causal ("DeDLOC Guide", Best Practices, Causal Mask Handling) with an
-// optional left window of W keys (axolotl-ringmaster README, Status:
-// sliding-window attention): query i sees keys i - W < j <= i; W = 0 means no
-// window. kSkip: no pair visible; kFull: every pair visible; kMask: mixed.
+// Which keys each query sees, in natural token positions. A query at position
+// i sees the keys lo(i) <= j <= hi(i); a key at position j is seen by the
+// queries imin(j) <= i <= imax(j). All four bounds are non-decreasing in the
+// position, so the visible pairs of any two tiles form a band. Without a table
+// they follow from the mask: causal ("DeDLOC Guide", Best Practices, Causal
+// Mask Handling) with an optional left window of W keys (axolotl-ringmaster
+// README, Status: sliding-window attention), query i seeing i - W < j <= i, or
+// no mask at all. With packed documents (the README's packing / varlen) a
+// per-token table {lo, hi, imin, imax} holds them (rm_varlen_bounds).
+struct MaskSpec {
+    const int4* tab;  // per-token bounds, or null
+    int S, causal, window;
+};
+
+// {lo(i), hi(i)}
+__device__ __forceinline__ int2 row_bounds(const MaskSpec& m, int i) {
+    if (m.tab) {
+        const int4 t = m.tab[i];
+        return make_int2(t.x, t.y);
+    }
+    return make_int2((m.causal && m.window) ? max(0, i - m.window + 1) : 0, m.causal ? i : m.S - 1);
+}
+
+// {imin(j), imax(j)}
+__device__ __forceinline__ int2 col_bounds(const MaskSpec& m, int j) {
+    if (m.tab) {
+        const int4 t = m.tab[j];
+        return make_int2(t.z, t.w);
+    }
+    return make_int2(m.causal ? j : 0,
+                     (m.causal && m.window) ? min(m.S - 1, j + m.window - 1) : m.S - 1);
+}
+
+// Class of a (128-query tile, 128-key tile) pair. kSkip: no pair visible;
+// kFull: every pair visible; kMask: mixed. From the query side: the bounds of
+// the tile's first row (f) and last row (l) against the key tile at kpos.
 enum : int { kSkip = 0, kMask = 1, kFull = 2 };
-__host__ __device__ __forceinline__ int band_tile_class(int causal, int window, int d) {
-    if (!causal) return kFull;
-    if (d < 0) return kSkip;                        // every key after every query
-    if (window == 0) return d == 0 ? kMask : kFull;
-    if (d >= window + 127) return kSkip;            // every key left of every window
-    return (d >= 128 && d <= window - 128) ? kFull : kMask;
+__device__ __forceinline__ int class_from_rows(int2 f, int2 l, int kpos) {
+    if (kpos > l.y || kpos + 127 < f.x) return kSkip;
+    return (kpos >= l.x && kpos + 127 <= f.y) ? kFull : kMask;
+}
+// The same pair from the key side: bounds of the key tile's first and last key
+// against the query tile at qpos.
+__device__ __forceinline__ int class_from_cols(int2 f, int2 l, int qpos) {
+    if (qpos > l.y || qpos + 127 < f.x) return kSkip;
+    return (qpos >= l.x && qpos + 127 <= f.y) ? kFull : kMask;
 }
 
 // ceil(x / 128) for any sign of x (the shift rounds toward minus infinity).

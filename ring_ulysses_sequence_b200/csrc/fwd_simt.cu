@@ -6,10 +6,10 @@
 // the key/value block of owner r = (i - t) mod P ("Sequence Parallelism III:
 // Ring Attention ...", duoan.github.io). Key tiles that the causal mask hides
 // entirely are skipped ("DeDLOC Guide", Best Practices, Causal Mask Handling),
-// and so are tiles left of every row's sliding window when one is set (query
-// i sees keys i - W < j <= i, axolotl-ringmaster README, Status); the online
-// softmax runs on across step boundaries, which is the merge of the steps'
-// partials ("DeDLOC Guide", section 3).
+// and so are tiles outside every row's sliding window or document when those
+// are set (axolotl-ringmaster README, Status); the online softmax runs on
+// across step boundaries, which is the merge of the steps' partials ("DeDLOC
+// Guide", section 3).
 #include "common.cuh"
 #include "internal.h"
 
@@ -30,7 +30,7 @@ struct F32Args {
     int H, Hkv, S, P, causal;
     float scale;
     RingLayout lay;
-    int window;  // causal left window in keys; 0 = none
+    MaskSpec mk;  // which keys each query sees
 };
 
 template <int D>
@@ -46,6 +46,9 @@ __global__ void __launch_bounds__(128) fwd_fp32_kernel(const __grid_constant__ F
     const int rank = s0 / L;
     const int qpos0 = a.lay.pos_of_slot(s0);
     const int qpos = qpos0 + row;
+    // key bounds of this row and of the block's first and last rows
+    const int2 rb = row_bounds(a.mk, qpos);
+    const int2 bf = row_bounds(a.mk, qpos0), bl = row_bounds(a.mk, qpos0 + kRows - 1);
 
     const float4* qrow =
         reinterpret_cast<const float4*>(a.q + ((static_cast<int64_t>(b) * a.H + h) * a.S + s0 + row) * D);
@@ -63,12 +66,9 @@ __global__ void __launch_bounds__(128) fwd_fp32_kernel(const __grid_constant__ F
         for (int u = 0; u < L / kKeys; ++u) {
             const int kslot = r * L + u * kKeys;
             const int kpos0 = a.lay.pos_of_slot(kslot);
-            if (a.causal && kpos0 > qpos0 + kRows - 1) continue;  // after every query
-            // window: tiles before every query's window are skipped; a tile is
-            // full when it is inside every query's window too
-            if (a.window && kpos0 + kKeys - 1 <= qpos0 - a.window) continue;
-            const bool full = !a.causal || (kpos0 + kKeys - 1 <= qpos0 &&
-                                            (a.window == 0 || kpos0 + a.window > qpos0 + kRows - 1));
+            // no row sees a key of this tile: skip; every row sees all of it: no mask
+            if (kpos0 > bl.y || kpos0 + kKeys - 1 < bf.x) continue;
+            const bool full = kpos0 >= bl.x && kpos0 + kKeys - 1 <= bf.y;
             __syncthreads();
             const float4* kg = reinterpret_cast<const float4*>(a.k + (kv_head + kslot) * D);
             const float4* vg = reinterpret_cast<const float4*>(a.v + (kv_head + kslot) * D);
@@ -94,9 +94,7 @@ __global__ void __launch_bounds__(128) fwd_fp32_kernel(const __grid_constant__ F
                     }
                     acc += __shfl_xor_sync(0xffffffffu, acc, 1);
                     acc *= a.scale;
-                    if (!full && (kpos0 + kb + jj > qpos ||
-                                  (a.window && kpos0 + kb + jj <= qpos - a.window)))
-                        acc = -INFINITY;
+                    if (!full && (kpos0 + kb + jj < rb.x || kpos0 + kb + jj > rb.y)) acc = -INFINITY;
                     s[jj] = acc;
                     mx = fmaxf(mx, acc);
                 }
@@ -143,7 +141,8 @@ cudaError_t launch_fwd_fp32(const AttnShape& sh, const float* q, const float* k,
     F32Args a{q, k, v, o, lse, sh.H, sh.Hkv, sh.S, sh.P, sh.causal, sh.scale,
               RingLayout{sh.S, sh.P, sh.S / sh.P, sh.zigzag ? sh.S / (2 * sh.P) : sh.S / sh.P,
                          sh.zigzag},
-              sh.causal ? sh.window : 0};
+              MaskSpec{static_cast<const int4*>(sh.bounds), sh.S, sh.causal,
+                       sh.causal ? sh.window : 0}};
     dim3 grid(sh.S / kRows, sh.H, sh.B);
     const size_t smem = 2 * static_cast<size_t>(kKeys) * sh.D * sizeof(float);
     if (sh.D == 64) {

@@ -63,8 +63,7 @@ struct TcArgs {
     unsigned* status;
     unsigned long long timeout_ns;
     int H, Hkv, S, P, causal, G;
-    int window;        // causal left window in keys; 0 = none
-    unsigned band;     // window, or 2^31 - 1 without one: the visible width of a row
+    MaskSpec mk;       // which keys each query sees
     int head_pair;     // 1: tiles are heads (h, h+1) at one slot; 0: one head, slots s, s+128
     int n_units;       // query units per head unit
     int n_head_units;  // B * (head_pair ? H / 2 : H)
@@ -107,18 +106,21 @@ __device__ __forceinline__ Item decode_item(const TcArgs& a, int w) {
 
 // Key tiles of an item in ring order: step t visits owner (rank - t) mod P.
 // An owner's block is one run (contiguous order) or two runs (zigzag: chunk r
-// then chunk 2P-1-r) of consecutive natural positions, so the tiles a causal
-// query tile can see form a prefix of each run, and with a window an interval
-// of it: O(1) work per tile returned, no division. kpos holds the natural
-// position of the tile last returned.
+// then chunk 2P-1-r) of consecutive natural positions. The keys that either
+// query tile can see form one interval [lo, hi] (the bounds are monotone), so
+// the tiles to visit in each run are an interval too: O(1) work per tile
+// returned, no division. kpos holds the natural position of the tile last
+// returned.
 struct KvIter {
-    const TcArgs* a;   // layout read from the kernel parameters, not copied
-    int rank, pos0, pos1, t, run, u, u_end, s0, p0, kpos;
-    __device__ __forceinline__ KvIter(const TcArgs& args, const Item& it)
-        : a(&args), rank(it.rank), pos0(it.pos0), pos1(it.pos1), t(0), run(-1), u(0), u_end(0),
-          s0(0), p0(0), kpos(0) {}
-    __device__ __forceinline__ bool next(int& kslot, int& c0, int& c1) {
-        const RingLayout& lay = a->lay;
+    int rank, lo, hi, t, run, u, u_end, s0, p0, kpos;
+    __device__ __forceinline__ KvIter(const TcArgs& a, const Item& it)
+        : rank(it.rank), t(0), run(-1), u(0), u_end(0), s0(0), p0(0), kpos(0) {
+        lo = min(row_bounds(a.mk, it.pos0).x, row_bounds(a.mk, it.pos1).x);
+        hi = max(row_bounds(a.mk, it.pos0 + kBM - 1).y, row_bounds(a.mk, it.pos1 + kBM - 1).y);
+    }
+    // `a` is the kernel's parameter block itself
+    __device__ __forceinline__ bool next(const TcArgs& a, int& kslot) {
+        const RingLayout& lay = a.lay;
         while (u >= u_end) {
             const int runs = lay.zigzag ? 2 : 1;
             if (++run == runs) {  // run starts at -1, so the first call opens run 0 of step 0
@@ -129,21 +131,13 @@ struct KvIter {
             const int ctiles = (lay.zigzag ? lay.c : lay.L) / kBN;
             s0 = r * lay.L + run * lay.c;
             p0 = lay.zigzag ? (run == 0 ? r * lay.c : (2 * lay.P - 1 - r) * lay.c) : r * lay.L;
-            u = 0;
-            u_end = ctiles;
-            if (a->causal) {
-                const int vis = ((max(pos0, pos1) - p0) >> 7) + 1;  // tiles at or before the query
-                u_end = min(ctiles, max(vis, 0));
-                // window: the first tile whose last key is inside the earliest
-                // row's window, kp + 127 > min(pos) - W
-                if (a->window) u = max(0, ceil_div128(min(pos0, pos1) - a->window - (kBN - 2) - p0));
-            }
+            // tiles whose keys meet [lo, hi]: p0 + 128 u <= hi and p0 + 128 u + 127 >= lo
+            u = max(0, ceil_div128(lo - (kBN - 1) - p0));
+            u_end = min(ctiles, max(((hi - p0) >> 7) + 1, 0));
         }
         kpos = p0 + u * kBN;
         kslot = s0 + u * kBN;
         ++u;
-        c0 = band_tile_class(a->causal, a->window, pos0 - kpos);
-        c1 = band_tile_class(a->causal, a->window, pos1 - kpos);
         return true;
     }
 };
@@ -235,8 +229,8 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
                                     bx * 64, row, smem_u32(&bars.q_full));
                 }
                 KvIter kv(a, it);
-                int kslot, c0, c1;
-                while (ok && kv.next(kslot, c0, c1)) {
+                int kslot;
+                while (ok && kv.next(a, kslot)) {
                     const int row = (it.b * a.Hkv + it.g) * a.S + kslot;
                     for (int which = 0; which < 2 && ok; ++which) {  // K then V
                         const int st = kv_iter % kStages;
@@ -272,9 +266,9 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
             for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x) {
                 const Item it = decode_item(a, w);
                 KvIter kv(a, it);
-                int ks, c0, c1;
-                bool have_cur = kv.next(ks, c0, c1);   // tile 0 (every item has one)
-                bool have_next = kv.next(ks, c0, c1);  // tile 1
+                int ks;
+                bool have_cur = kv.next(a, ks);   // tile 0 (every item has one)
+                bool have_next = kv.next(a, ks);  // tile 1
                 ok = mbar_wait(smem_u32(&bars.q_full), q_iter & 1, wd);
                 if (!ok) break;
                 ++q_iter;
@@ -291,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
                 umma_commit(smem_u32(&bars.kv_empty[stK]));
                 if (!have_next) umma_commit(smem_u32(&bars.q_empty));
                 for (int j = 0; have_cur && ok; ++j) {
-                    const bool have_next2 = have_next && kv.next(ks, c0, c1);  // tile j + 2
+                    const bool have_next2 = have_next && kv.next(a, ks);  // tile j + 2
                     const uint32_t stV = kv_iter % kStages;
                     ok = mbar_wait(smem_u32(&bars.kv_full[stV]), (kv_iter / kStages) & 1, wd);
                     if (!ok) break;
@@ -349,9 +343,11 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
             const Item it = decode_item(a, w);
             float m = -INFINITY, l = 0.f;
             KvIter kv(a, it);
-            int kslot, c0, c1, j = 0;
-            while (ok && kv.next(kslot, c0, c1)) {
-                const int cls = x ? c1 : c0;
+            const int qpos = x ? it.pos1 : it.pos0;
+            const int2 bf = row_bounds(a.mk, qpos), bl = row_bounds(a.mk, qpos + kBM - 1);
+            int kslot, j = 0;
+            while (ok && kv.next(a, kslot)) {
+                const int cls = class_from_rows(bf, bl, kv.kpos);
                 ok = mbar_wait(smem_u32(&bars.s_full[x]), (s_cnt++) & 1, wd);
                 if (!ok) break;
                 tc_fence_after();
@@ -371,11 +367,13 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
 #pragma unroll
                     for (int c = 0; c < 64; ++c) s[64 + c] = __uint_as_float(raw[c]);
                     if (cls == kMask) {
-                        // key column c is visible iff 0 <= hi - c < band
-                        const int hi = r + (x ? it.pos1 : it.pos0) - kv.kpos;
+                        // key column c is visible iff lo(i) <= kpos + c <= hi(i)
+                        const int2 rb = row_bounds(a.mk, qpos + r);
+                        const int lo = rb.x - kv.kpos;
+                        const unsigned w = static_cast<unsigned>(rb.y - rb.x);
 #pragma unroll
                         for (int c = 0; c < 128; ++c)
-                            if (static_cast<unsigned>(hi - c) >= a.band) s[c] = -INFINITY;
+                            if (static_cast<unsigned>(c - lo) > w) s[c] = -INFINITY;
                     }
                     float mx = s[0];
 #pragma unroll
@@ -389,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
                         m = m_new;
                         rescale_o = j > 0;
                     }
-                    // m stays -inf while a windowed row has seen no key: p = 0 then
+                    // m stays -inf while a row has seen no key of its band: p = 0 then
                     const float neg = m == -INFINITY ? 0.f : -m * sl2;
                     float rs = 0.f;
                     uint32_t pk[32];
@@ -480,8 +478,7 @@ cudaError_t launch_fwd_tc(const AttnShape& sh, const void* q, const void* k, con
     a.P = sh.P;
     a.causal = sh.causal;
     a.G = sh.H / sh.Hkv;
-    a.window = sh.causal ? sh.window : 0;
-    a.band = a.window ? static_cast<unsigned>(a.window) : 0x7fffffffu;
+    a.mk = MaskSpec{static_cast<const int4*>(sh.bounds), sh.S, sh.causal, sh.causal ? sh.window : 0};
     a.head_pair = (a.G % 2 == 0) ? 1 : 0;
     a.n_units = a.head_pair ? sh.S / kBM : sh.S / (2 * kBM);
     a.n_head_units = sh.B * (a.head_pair ? sh.H / 2 : sh.H);

@@ -19,7 +19,8 @@ struct LaunchCtx {
 struct AttnShape {
     int B, H, Hkv, S, D, P, causal, zigzag;
     float scale;
-    int window;  // causal left window in keys (query i sees i - window < j <= i); 0 = none
+    int window;            // causal left window in keys (query i sees i - window < j <= i); 0 = none
+    const void* bounds;    // per-token int4 {lo, hi, imin, imax} of packed documents, or null
 };
 
 // Forward, bf16, tcgen05 tensor cores (fwd_tc.cu).
@@ -46,5 +47,9 @@ cudaError_t launch_seq_reorder(const void* src, void* dst, int BH, int S, int D,
 cudaError_t launch_lse_merge(float* o_acc, float* lse_acc, const float* o_part,
                              const float* lse_part, int64_t rows, int D, const LaunchCtx& ctx);
 cudaError_t launch_watchdog_selftest(const LaunchCtx& ctx);
+// Per-token bounds of packed documents into `table` (S int4); cu_dev holds
+// n_docs + 1 checked boundaries in device memory.
+cudaError_t launch_varlen_bounds(const int* cu_dev, int n_docs, int S, int causal, int window,
+                                 void* table, const LaunchCtx& ctx);
 
 }  // namespace rm

@@ -189,7 +189,44 @@ int pick_vec(int64_t row_bytes, const void* a, const void* b) {
     return 1;
 }
 
+// Per-token visibility bounds of packed documents (axolotl-ringmaster README,
+// Status: packing / varlen). cu[0..n] rises from 0 to S (checked on the host);
+// token i lies in document d with cu[d] <= i < cu[d+1] (the last such d when
+// empty documents repeat a boundary). A query sees the keys of its own
+// document, up to itself when causal and not before i - W + 1 with a window:
+//   lo(i) = max(cu[d], i - W + 1),  hi(i) = causal ? i : cu[d+1] - 1;
+// and a key j is seen by the queries
+//   imin(j) = causal ? j : cu[d],  imax(j) = min(cu[d+1] - 1, j + W - 1).
+__global__ void __launch_bounds__(256) varlen_bounds_kernel(const int* __restrict__ cu, int n_docs,
+                                                            int S, int causal, int window,
+                                                            int4* __restrict__ tab) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < S; i += gridDim.x * blockDim.x) {
+        int a = 0, b = n_docs - 1;  // largest d in [0, n) with cu[d] <= i
+        while (a < b) {
+            const int mid = (a + b + 1) >> 1;
+            if (cu[mid] <= i) a = mid;
+            else b = mid - 1;
+        }
+        const int ds = cu[a], de = cu[a + 1];
+        int lo = ds, imax = de - 1;
+        if (causal && window) {
+            lo = max(lo, i - window + 1);
+            imax = min(imax, i + window - 1);
+        }
+        tab[i] = make_int4(lo, causal ? i : de - 1, causal ? i : ds, imax);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_varlen_bounds(const int* cu_dev, int n_docs, int S, int causal, int window,
+                                 void* table, const LaunchCtx& ctx) {
+    const int threads = 256;
+    const int blocks = std::max(1, std::min((S + threads - 1) / threads, ctx.num_sms * 8));
+    varlen_bounds_kernel<<<blocks, threads, 0, ctx.stream>>>(cu_dev, n_docs, S, causal, window,
+                                                             static_cast<int4*>(table));
+    return cudaGetLastError();
+}
 
 cudaError_t launch_ulysses_permute(const PermuteTensor* t, int ntensors, int B, int S, int D,
                                    int elem_bytes, int head_to_seq, const LaunchCtx& ctx) {

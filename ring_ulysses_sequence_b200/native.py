@@ -23,11 +23,17 @@ SIGNATURES = {
     "rm_ring_attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "rm_ring_attn_fwd_window": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                                      _f, _vp]),
+    "rm_varlen_bounds_size": (_sz, [_i, _i]),
+    "rm_varlen_bounds": (_i, [_vp, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "rm_ring_attn_fwd_varlen": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
+                                     _f, _vp]),
     "rm_ring_attn_bwd_workspace_size": (_sz, [_i, _i, _i]),
     "rm_ring_attn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                               _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "rm_ring_attn_bwd_window": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                                      _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
+    "rm_ring_attn_bwd_varlen": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                                     _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "rm_ring_attn_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                       _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "rm_lse_merge": (_i, [_vp, _vp, _vp, _vp, _i64, _i, _vp]),
@@ -108,6 +114,23 @@ def rm_ring_attn_fwd_window(q, k, v, o, lse, B, H, Hkv, S, D, P, window, order, 
                  P, window, order, dtype, scale, _s(stream))
 
 
+def rm_varlen_bounds_size(S, n_docs):
+    return int(lib().rm_varlen_bounds_size(S, n_docs))
+
+
+def rm_varlen_bounds(cu_seqlens, n_docs, S, causal, window, bounds, bounds_bytes, stream=None):
+    """cu_seqlens: a sequence of n_docs + 1 host integers."""
+    arr = (ctypes.c_int * (n_docs + 1))(*[int(x) for x in cu_seqlens])
+    return _call("rm_varlen_bounds", ctypes.cast(arr, ctypes.c_void_p), n_docs, S, int(causal),
+                 window, _p(bounds), bounds_bytes, _s(stream))
+
+
+def rm_ring_attn_fwd_varlen(q, k, v, o, lse, bounds, B, H, Hkv, S, D, P, order, dtype, scale,
+                            stream=None):
+    return _call("rm_ring_attn_fwd_varlen", _p(q), _p(k), _p(v), _p(o), _p(lse), _p(bounds), B,
+                 H, Hkv, S, D, P, order, dtype, scale, _s(stream))
+
+
 def rm_ring_attn_bwd_workspace_size(B, H, S):
     return int(lib().rm_ring_attn_bwd_workspace_size(B, H, S))
 
@@ -124,6 +147,13 @@ def rm_ring_attn_bwd_window(q, k, v, o, lse, dout, dq, dk, dv, workspace, worksp
     return _call("rm_ring_attn_bwd_window", _p(q), _p(k), _p(v), _p(o), _p(lse), _p(dout),
                  _p(dq), _p(dk), _p(dv), _p(workspace), workspace_bytes, B, H, Hkv, S, D, P,
                  window, order, dtype, scale, _s(stream))
+
+
+def rm_ring_attn_bwd_varlen(q, k, v, o, lse, dout, dq, dk, dv, bounds, workspace, workspace_bytes,
+                            B, H, Hkv, S, D, P, order, dtype, scale, stream=None):
+    return _call("rm_ring_attn_bwd_varlen", _p(q), _p(k), _p(v), _p(o), _p(lse), _p(dout),
+                 _p(dq), _p(dk), _p(dv), _p(bounds), _p(workspace), workspace_bytes, B, H, Hkv,
+                 S, D, P, order, dtype, scale, _s(stream))
 
 
 def rm_ring_attn_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, H, Hkv, S, D, P, causal,

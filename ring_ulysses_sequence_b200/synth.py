@@ -33,6 +33,7 @@ class Workload:
     ulysses: int = 1      # U; the ring size is P
     backward: bool = False
     window: int = 0       # causal sliding window in keys (query i sees i-W < j <= i); 0 = none
+    cu_seqlens: tuple = ()  # packed document boundaries (natural positions, 0 .. S); () = none
     notes: str = field(default="", compare=False)
 
     @property
@@ -46,7 +47,12 @@ class Workload:
 
     def fwd_flops(self) -> float:
         """Algorithmic forward FLOPs: 4 B H S^2 D, halved when causal; with a
-        window, 4 B H D times the number of visible (query, key) pairs."""
+        window or packed documents, 4 B H D times the number of visible
+        (query, key) pairs."""
+        if self.cu_seqlens:
+            lens = np.diff(np.asarray(self.cu_seqlens, dtype=np.int64))
+            pairs = int((lens * (lens + 1) // 2).sum()) if self.causal else int((lens * lens).sum())
+            return 4.0 * self.B * self.H * self.D * pairs
         if self.causal and 0 < self.window < self.S:
             W, S = self.window, self.S
             pairs = W * (W + 1) // 2 + (S - W) * W
@@ -57,6 +63,16 @@ class Workload:
     def bwd_flops(self) -> float:
         """Algorithmic backward FLOPs: 2.5x the forward (five products vs two)."""
         return 2.5 * self.fwd_flops()
+
+
+def packed_boundaries(S: int, seed: int, lo: int = 512, hi: int = 8192) -> list:
+    """Document boundaries 0 = cu[0] < ... < cu[n] = S: lengths drawn uniformly
+    from [lo, hi] with a seeded generator, the last document cut at S."""
+    rng = np.random.default_rng(seed)
+    cu = [0]
+    while cu[-1] < S:
+        cu.append(min(S, cu[-1] + int(rng.integers(lo, hi + 1))))
+    return cu
 
 
 WORKLOADS = {
@@ -77,6 +93,11 @@ WORKLOADS = {
     "ring_fwd_bf16_S32k_gqa_causal_zigzag_window4k": Workload(
         "ring_fwd_bf16_S32k_gqa_causal_zigzag_window4k", 1, 32, 8, 32768, 128, 8, "zigzag", True,
         torch.bfloat16, 5, 0.5, window=4096),
+    # The same layer over packed documents of seeded lengths (512 to 8192
+    # tokens): attention stays inside each document.
+    "ring_fwd_bf16_S32k_gqa_causal_zigzag_packed": Workload(
+        "ring_fwd_bf16_S32k_gqa_causal_zigzag_packed", 1, 32, 8, 32768, 128, 8, "zigzag", True,
+        torch.bfloat16, 6, 0.5, cu_seqlens=tuple(packed_boundaries(32768, 6))),
     # Ulysses x Ring: 4 x 4 mesh over 131072 tokens, sequence-sharded input
     # [16 shards, 8192 tokens, heads, 128].
     "usp_fwd_bf16_S128k_u4r4": Workload("usp_fwd_bf16_S128k_u4r4", 1, 32, 8, 131072, 128, 4,

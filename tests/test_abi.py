@@ -29,6 +29,7 @@ def test_header_declares_the_path():
     fns = header_functions()
     for name in ("rm_ring_attn_fwd", "rm_ring_attn_bwd", "rm_ring_attn_bwd_workspace_size",
                  "rm_ring_attn_fwd_window", "rm_ring_attn_bwd_window",
+                 "rm_varlen_bounds", "rm_ring_attn_fwd_varlen", "rm_ring_attn_bwd_varlen",
                  "rm_lse_merge", "rm_ulysses_permute", "rm_ulysses_permute_qkv",
                  "rm_seq_reorder", "rm_check_device_status", "rm_status_string"):
         assert name in fns
@@ -124,6 +125,30 @@ def test_window_calls_reach_the_device_without_gpu(lib):
                                        None) == 3
     assert lib.rm_ring_attn_fwd_window(A, A, A, A, A, 1, 4, 2, 1024, 64, 4, 5000, 0, 1, 0.125,
                                        None) == 3
+
+
+def test_varlen_validation(lib):
+    import ctypes
+    def cu(*xs):
+        return (ctypes.c_int * len(xs))(*xs)
+    size = lib.rm_varlen_bounds_size(1024, 3)
+    assert size >= 1024 * 16 + 16 and size % 256 == 0
+    assert lib.rm_varlen_bounds_size(0, 3) == 0
+    B = 1 << 20  # 256-byte aligned fake buffer, never touched: validation comes first
+    ok = cu(0, 100, 700, 1024)
+    assert lib.rm_varlen_bounds(cu(0, 700, 100, 1024), 3, 1024, 1, 0, B, size, None) == 1  # falls
+    assert lib.rm_varlen_bounds(cu(5, 100, 700, 1024), 3, 1024, 1, 0, B, size, None) == 1  # not 0
+    assert lib.rm_varlen_bounds(cu(0, 100, 700, 1000), 3, 1024, 1, 0, B, size, None) == 1  # not S
+    assert lib.rm_varlen_bounds(ok, 3, 1024, 0, 16, B, size, None) == 1    # window needs causal
+    assert lib.rm_varlen_bounds(ok, 3, 1024, 1, 0, B, size - 256, None) == 1  # too small
+    assert lib.rm_varlen_bounds(ok, 3, 1024, 1, 0, B + 16, size, None) == 1   # misaligned
+    assert lib.rm_varlen_bounds(ok, 0, 1024, 1, 0, B, size, None) == 1
+    assert lib.rm_varlen_bounds(cu(0, 0), 1, 0, 1, 0, None, 0, None) == 0     # empty: no-op
+    # the attention calls need a table
+    assert lib.rm_ring_attn_fwd_varlen(A, A, A, A, A, None, 1, 4, 2, 1024, 128, 4, 1, 0, 0.088,
+                                       None) == 1
+    assert lib.rm_ring_attn_fwd_varlen(A, A, A, A, A, B, 1, 4, 2, 1004, 128, 4, 1, 0, 0.088,
+                                       None) == 1
 
 
 def test_layout_validation(lib):
