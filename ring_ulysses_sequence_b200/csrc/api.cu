@@ -10,6 +10,15 @@ namespace rm {
 
 // Device status word: bit 0 = a bounded wait ran out. One copy per device.
 __device__ unsigned g_status_word;
+// Work-item counters of the persistent kernels (one slot per launch in flight).
+__device__ int g_work_counters[kWorkSlots];
+static std::atomic<uint32_t> g_work_seq{0};
+
+cudaError_t next_work_counter(const LaunchCtx& ctx, int** counter) {
+    int* c = ctx.work_counters + (g_work_seq.fetch_add(1) % kWorkSlots);
+    *counter = c;
+    return cudaMemsetAsync(c, 0, sizeof(int), ctx.stream);
+}
 
 static thread_local int t_last_cuda_error = 0;
 static std::atomic<uint64_t> g_watchdog_ns{2000000000ull};
@@ -26,6 +35,7 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 static rm_status get_ctx(cudaStream_t stream, LaunchCtx* ctx) {
     static std::mutex mu;
     static unsigned* word_addr[128] = {};
+    static int* counters_addr[128] = {};
     static int sms[128] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -37,6 +47,10 @@ static rm_status get_ctx(cudaStream_t stream, LaunchCtx* ctx) {
             void* p = nullptr;
             e = cudaGetSymbolAddress(&p, g_status_word);
             if (e != cudaSuccess) return cuda_fail(e);
+            void* pc = nullptr;
+            e = cudaGetSymbolAddress(&pc, g_work_counters);
+            if (e != cudaSuccess) return cuda_fail(e);
+            counters_addr[dev] = static_cast<int*>(pc);
             int n = 0;
             e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
             if (e != cudaSuccess) return cuda_fail(e);
@@ -44,6 +58,7 @@ static rm_status get_ctx(cudaStream_t stream, LaunchCtx* ctx) {
             word_addr[dev] = static_cast<unsigned*>(p);
         }
         ctx->status_word = word_addr[dev];
+        ctx->work_counters = counters_addr[dev];
         ctx->num_sms = sms[dev];
     }
     ctx->watchdog_ns = g_watchdog_ns.load();

@@ -53,7 +53,7 @@ struct Cfg {
     static constexpr int kQOff = 0;
     static constexpr int kKVOff = 2 * kTileBytes;
     static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
-    static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + barriers + alignment slack
+    static constexpr int kSmemBytes = kBarOff + 512 + 1024;  // + barriers + alignment slack
 };
 
 struct TcArgs {
@@ -61,6 +61,7 @@ struct TcArgs {
     void* o;
     float* lse;
     unsigned* status;
+    int* work;         // this launch's work-item counter
     unsigned long long timeout_ns;
     int H, Hkv, S, P, causal, G;
     MaskSpec mk;       // which keys each query sees
@@ -142,7 +143,12 @@ struct KvIter {
     }
 };
 
+constexpr int kItemRing = 4;  // work items the producer may claim ahead of the consumers
+constexpr int kItemReaders = 9;  // the MMA thread and one lane of each softmax warp
+
 struct Bars {
+    uint64_t item_full[kItemRing], item_empty[kItemRing];
+    int item_id[kItemRing];
     uint64_t q_full, q_empty, drain;
     uint64_t kv_full[kStages], kv_empty[kStages];
     uint64_t s_full[2], p_full[2], o_full[2];
@@ -172,6 +178,43 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint3
                 (accumulate || k > 0) ? 1u : 0u);
 }
 
+// Work items are claimed dynamically: the producer thread takes the next item
+// index from the launch's counter (so a CTA that finishes early takes more
+// work) and publishes it in a ring of kItemRing slots; the MMA thread and the
+// softmax warps read the k-th claimed index from slot k % kItemRing. An index
+// >= n_items means no more work.
+__device__ __forceinline__ bool claim_item(const TcArgs& a, Bars& bars, uint32_t k, int& w,
+                                           const Watchdog& wd) {
+    const int slot = k % kItemRing;
+    if (k >= kItemRing &&
+        !mbar_wait(smem_u32(&bars.item_empty[slot]), (k / kItemRing - 1) & 1, wd))
+        return false;
+    w = atomicAdd(a.work, 1);
+    bars.item_id[slot] = w;
+    mbar_arrive(smem_u32(&bars.item_full[slot]));  // release: the index is visible first
+    return true;
+}
+
+// Reads the k-th claimed index. A whole warp calls it with `warp_wide` set and
+// its lane 0 releases the slot once every lane has read it; a single thread
+// (the MMA issuer, whose other lanes do not take part) calls it with
+// `warp_wide` clear and releases the slot itself.
+__device__ __forceinline__ bool read_item(Bars& bars, uint32_t k, int& w, bool warp_wide,
+                                          const Watchdog& wd) {
+    const int slot = k % kItemRing;
+    bool ok = mbar_wait(smem_u32(&bars.item_full[slot]), (k / kItemRing) & 1, wd);
+    if (warp_wide) ok = __all_sync(0xffffffffu, ok);  // the lanes leave together
+    if (!ok) return false;
+    w = *reinterpret_cast<volatile int*>(&bars.item_id[slot]);
+    if (warp_wide) {
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&bars.item_empty[slot]));
+    } else {
+        mbar_arrive(smem_u32(&bars.item_empty[slot]));
+    }
+    return true;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_constant__ TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -184,6 +227,10 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
 
     if (threadIdx.x == 0) {
         bars.abort_flag = 0;
+        for (int i = 0; i < kItemRing; ++i) {
+            mbar_init(smem_u32(&bars.item_full[i]), 1);
+            mbar_init(smem_u32(&bars.item_empty[i]), kItemReaders);
+        }
         mbar_init(smem_u32(&bars.q_full), 1);
         mbar_init(smem_u32(&bars.q_empty), 1);
         mbar_init(smem_u32(&bars.drain), 1);
@@ -216,7 +263,10 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
             prefetch_tmap(&a.tm_v);
             uint32_t q_iter = 0, kv_iter = 0;
             bool ok = true;
-            for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x) {
+            for (uint32_t k = 0; ok; ++k) {
+                int w;
+                ok = claim_item(a, bars, k, w, wd);
+                if (!ok || w >= a.n_items) break;
                 const Item it = decode_item(a, w);
                 if (q_iter > 0) ok = mbar_wait(smem_u32(&bars.q_empty), (q_iter - 1) & 1, wd);
                 if (!ok) break;
@@ -263,7 +313,10 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
             const uint32_t tO[2] = {tmem + 256, tmem + 384};
             uint32_t q_iter = 0, kv_iter = 0, p_cnt[2] = {0, 0};
             bool ok = true;
-            for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x) {
+            for (uint32_t k = 0; ok; ++k) {
+                int w;
+                ok = read_item(bars, k, w, false, wd);
+                if (!ok || w >= a.n_items) break;
                 const Item it = decode_item(a, w);
                 KvIter kv(a, it);
                 int ks;
@@ -339,7 +392,10 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
         const float sl2 = a.scale_log2;
         uint32_t s_cnt = 0, o_cnt = 0;
         bool ok = true;
-        for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x) {
+        for (uint32_t k = 0; ok; ++k) {
+            int w;
+            ok = read_item(bars, k, w, true, wd);
+            if (!ok || w >= a.n_items) break;
             const Item it = decode_item(a, w);
             float m = -INFINITY, l = 0.f;
             KvIter kv(a, it);
@@ -471,6 +527,7 @@ cudaError_t launch_fwd_tc(const AttnShape& sh, const void* q, const void* k, con
     a.o = o;
     a.lse = lse;
     a.status = ctx.status_word;
+    if ((e = next_work_counter(ctx, &a.work)) != cudaSuccess) return e;
     a.timeout_ns = ctx.watchdog_ns;
     a.H = sh.H;
     a.Hkv = sh.Hkv;

@@ -11,6 +11,7 @@ namespace rm {
 // Per-launch context: device status word, watchdog limit, device properties.
 struct LaunchCtx {
     unsigned* status_word;   // device address of the status word
+    int* work_counters;      // device address of kWorkSlots dynamic-schedule counters
     uint64_t watchdog_ns;
     int num_sms;
     cudaStream_t stream;
@@ -22,6 +23,14 @@ struct AttnShape {
     int window;            // causal left window in keys (query i sees i - window < j <= i); 0 = none
     const void* bounds;    // per-token int4 {lo, hi, imin, imax} of packed documents, or null
 };
+
+// Dynamic work distribution: a persistent kernel's CTAs take work items from a
+// counter in device memory. Each launch uses its own counter slot (rotating
+// over kWorkSlots), zeroed on the launch's stream just before it; at most
+// kWorkSlots launches may be in flight at once.
+constexpr int kWorkSlots = 256;
+// Zeroes a fresh counter slot on ctx.stream and returns its address.
+cudaError_t next_work_counter(const LaunchCtx& ctx, int** counter);
 
 // Forward, bf16, tcgen05 tensor cores (fwd_tc.cu).
 cudaError_t launch_fwd_tc(const AttnShape& sh, const void* q, const void* k, const void* v,
