@@ -68,6 +68,7 @@ struct BwdArgs {
     float* dk;
     float* dv;
     unsigned* status;
+    int* work;       // this launch's work-item counter
     unsigned long long timeout_ns;
     int B, H, Hkv, S, P, causal, G, n_items;
     MaskSpec mk;     // which keys each query sees
@@ -75,13 +76,17 @@ struct BwdArgs {
     RingLayout lay;
 };
 
+constexpr int kItemReaders = 9;  // the MMA thread and one lane of each compute warp
+
 struct Bars {
+    ItemRing items;  // work items claimed by the producer (dynamic distribution)
     uint64_t res_full, res_empty, drain, acc_full;
     uint64_t st_full[kStages], st_empty[kStages];
     uint64_t s_full, p_full;
     uint32_t tmem_base;
     int abort_flag;
 };
+static_assert(sizeof(Bars) <= 256, "barrier block");
 
 // -------------------------------------------------------------------- dK / dV
 
@@ -204,6 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
 
     if (threadIdx.x == 0) {
         bars.abort_flag = 0;
+        item_ring_init(bars.items, kItemReaders);
         mbar_init(smem_u32(&bars.res_full), 1);
         mbar_init(smem_u32(&bars.res_empty), 1);
         mbar_init(smem_u32(&bars.drain), 1);
@@ -234,7 +240,10 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
             prefetch_tmap(&a.tm_do);
             uint32_t items = 0, fills = 0;
             bool ok = true;
-            for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x, ++items) {
+            for (uint32_t k = 0; ok; ++k, ++items) {
+                int w;
+                ok = item_claim(bars.items, a.work, k, w, wd);
+                if (!ok || w >= a.n_items) break;
                 const KvItem it = decode_kv_item(a, w);
                 if (items > 0) ok = mbar_wait(smem_u32(&bars.res_empty), (items - 1) & 1, wd);
                 if (!ok) break;
@@ -277,7 +286,10 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
             const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 384;
             uint32_t items = 0, uses = 0, p_cnt = 0;
             bool ok = true;
-            for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x, ++items) {
+            for (uint32_t k = 0; ok; ++k, ++items) {
+                int w;
+                ok = item_read(bars.items, k, w, false, wd);
+                if (!ok || w >= a.n_items) break;
                 const KvItem it = decode_kv_item(a, w);
                 QIter qi(a, it);
                 int qh, qs, qc;
@@ -324,7 +336,10 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
         const float sl2 = a.scale_log2;
         uint32_t uses = 0, s_cnt = 0, items = 0;
         bool ok = true;
-        for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x, ++items) {
+        for (uint32_t k = 0; ok; ++k, ++items) {
+            int w;
+            ok = item_read(bars.items, k, w, true, wd);
+            if (!ok || w >= a.n_items) break;
             const KvItem it = decode_kv_item(a, w);
             QIter qi(a, it);
             int h, qslot, cls;
@@ -477,6 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
 
     if (threadIdx.x == 0) {
         bars.abort_flag = 0;
+        item_ring_init(bars.items, kItemReaders);
         mbar_init(smem_u32(&bars.res_full), 1);
         mbar_init(smem_u32(&bars.res_empty), 1);
         mbar_init(smem_u32(&bars.drain), 1);
@@ -507,7 +523,10 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
             prefetch_tmap(&a.tm_do);
             uint32_t items = 0, fills = 0;
             bool ok = true;
-            for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x, ++items) {
+            for (uint32_t k = 0; ok; ++k, ++items) {
+                int w;
+                ok = item_claim(bars.items, a.work, k, w, wd);
+                if (!ok || w >= a.n_items) break;
                 const QItem it = decode_q_item(a, w);
                 if (items > 0) ok = mbar_wait(smem_u32(&bars.res_empty), (items - 1) & 1, wd);
                 if (!ok) break;
@@ -548,7 +567,10 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
             const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
             uint32_t items = 0, uses = 0, p_cnt = 0;
             bool ok = true;
-            for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x, ++items) {
+            for (uint32_t k = 0; ok; ++k, ++items) {
+                int w;
+                ok = item_read(bars.items, k, w, false, wd);
+                if (!ok || w >= a.n_items) break;
                 const QItem it = decode_q_item(a, w);
                 KIter ki(a, it);
                 int ks, kc;
@@ -593,7 +615,10 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
         const float sl2 = a.scale_log2;
         uint32_t s_cnt = 0, items = 0;
         bool ok = true;
-        for (int w = blockIdx.x; ok && w < a.n_items; w += gridDim.x, ++items) {
+        for (uint32_t k = 0; ok; ++k, ++items) {
+            int w;
+            ok = item_read(bars.items, k, w, true, wd);
+            if (!ok || w >= a.n_items) break;
             const QItem it = decode_q_item(a, w);
             const int64_t qrow = (static_cast<int64_t>(it.b) * a.H + it.h) * a.S + it.slot + r;
             const float lse2 = a.lse[qrow] * kLog2e;
@@ -700,6 +725,7 @@ cudaError_t launch_bwd_d(const AttnShape& sh, const BwdArgs& base, const void* o
 
     BwdArgs a = base;
     a.n_items = sh.B * sh.Hkv * (sh.S / kT);
+    if ((e = next_work_counter(ctx, &a.work)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(ring_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   BCfg<D>::kSmemKV)) != cudaSuccess)
         return e;
@@ -707,6 +733,7 @@ cudaError_t launch_bwd_d(const AttnShape& sh, const BwdArgs& base, const void* o
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     a.n_items = sh.B * sh.H * (sh.S / kT);
+    if ((e = next_work_counter(ctx, &a.work)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(ring_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   BCfg<D>::kSmemQ)) != cudaSuccess)
         return e;

@@ -166,6 +166,61 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
 }
 
 // ---------------------------------------------------------------------------
+// Dynamic work distribution inside a persistent CTA. The producer thread takes
+// the next work-item index from the launch's counter in device memory (so a CTA
+// that finishes early takes more work) and publishes it in a ring of
+// kItemRing slots; the other roles read the k-th claimed index from slot
+// k % kItemRing. An index >= the item count means no more work.
+// ---------------------------------------------------------------------------
+
+constexpr int kItemRing = 4;
+
+struct ItemRing {
+    uint64_t full[kItemRing], empty[kItemRing];
+    int id[kItemRing];
+};
+
+// readers: the number of arrivals that release a slot.
+__device__ __forceinline__ void item_ring_init(ItemRing& r, int readers) {
+    for (int i = 0; i < kItemRing; ++i) {
+        mbar_init(smem_u32(&r.full[i]), 1);
+        mbar_init(smem_u32(&r.empty[i]), readers);
+    }
+}
+
+// Claims the k-th item of this CTA (one thread).
+__device__ __forceinline__ bool item_claim(ItemRing& r, int* counter, uint32_t k, int& w,
+                                           const Watchdog& wd) {
+    const int slot = k % kItemRing;
+    if (k >= kItemRing && !mbar_wait(smem_u32(&r.empty[slot]), (k / kItemRing - 1) & 1, wd))
+        return false;
+    w = atomicAdd(counter, 1);
+    r.id[slot] = w;
+    mbar_arrive(smem_u32(&r.full[slot]));  // release: the index is visible first
+    return true;
+}
+
+// Reads the k-th claimed item. A whole warp calls it with `warp_wide` set and
+// its lane 0 releases the slot once every lane has read it; a single thread
+// whose other lanes do not take part calls it with `warp_wide` clear and
+// releases the slot itself (a warp-wide sync there would wait forever).
+__device__ __forceinline__ bool item_read(ItemRing& r, uint32_t k, int& w, bool warp_wide,
+                                          const Watchdog& wd) {
+    const int slot = k % kItemRing;
+    bool ok = mbar_wait(smem_u32(&r.full[slot]), (k / kItemRing) & 1, wd);
+    if (warp_wide) ok = __all_sync(0xffffffffu, ok);  // the lanes leave together
+    if (!ok) return false;
+    w = *reinterpret_cast<volatile int*>(&r.id[slot]);
+    if (warp_wide) {
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&r.empty[slot]));
+    } else {
+        mbar_arrive(smem_u32(&r.empty[slot]));
+    }
+    return true;
+}
+
+// ---------------------------------------------------------------------------
 // TMA (no multicast anywhere in this library)
 // ---------------------------------------------------------------------------
 

@@ -143,18 +143,17 @@ struct KvIter {
     }
 };
 
-constexpr int kItemRing = 4;  // work items the producer may claim ahead of the consumers
 constexpr int kItemReaders = 9;  // the MMA thread and one lane of each softmax warp
 
 struct Bars {
-    uint64_t item_full[kItemRing], item_empty[kItemRing];
-    int item_id[kItemRing];
+    ItemRing items;  // work items claimed by the producer (dynamic distribution)
     uint64_t q_full, q_empty, drain;
     uint64_t kv_full[kStages], kv_empty[kStages];
     uint64_t s_full[2], p_full[2], o_full[2];
     uint32_t tmem_base;
     int abort_flag;
 };
+static_assert(sizeof(Bars) <= 512, "barrier block");
 
 template <int D>
 __device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_smem, uint32_t k_smem) {
@@ -178,43 +177,6 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint3
                 (accumulate || k > 0) ? 1u : 0u);
 }
 
-// Work items are claimed dynamically: the producer thread takes the next item
-// index from the launch's counter (so a CTA that finishes early takes more
-// work) and publishes it in a ring of kItemRing slots; the MMA thread and the
-// softmax warps read the k-th claimed index from slot k % kItemRing. An index
-// >= n_items means no more work.
-__device__ __forceinline__ bool claim_item(const TcArgs& a, Bars& bars, uint32_t k, int& w,
-                                           const Watchdog& wd) {
-    const int slot = k % kItemRing;
-    if (k >= kItemRing &&
-        !mbar_wait(smem_u32(&bars.item_empty[slot]), (k / kItemRing - 1) & 1, wd))
-        return false;
-    w = atomicAdd(a.work, 1);
-    bars.item_id[slot] = w;
-    mbar_arrive(smem_u32(&bars.item_full[slot]));  // release: the index is visible first
-    return true;
-}
-
-// Reads the k-th claimed index. A whole warp calls it with `warp_wide` set and
-// its lane 0 releases the slot once every lane has read it; a single thread
-// (the MMA issuer, whose other lanes do not take part) calls it with
-// `warp_wide` clear and releases the slot itself.
-__device__ __forceinline__ bool read_item(Bars& bars, uint32_t k, int& w, bool warp_wide,
-                                          const Watchdog& wd) {
-    const int slot = k % kItemRing;
-    bool ok = mbar_wait(smem_u32(&bars.item_full[slot]), (k / kItemRing) & 1, wd);
-    if (warp_wide) ok = __all_sync(0xffffffffu, ok);  // the lanes leave together
-    if (!ok) return false;
-    w = *reinterpret_cast<volatile int*>(&bars.item_id[slot]);
-    if (warp_wide) {
-        __syncwarp();
-        if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&bars.item_empty[slot]));
-    } else {
-        mbar_arrive(smem_u32(&bars.item_empty[slot]));
-    }
-    return true;
-}
-
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_constant__ TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -227,10 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
 
     if (threadIdx.x == 0) {
         bars.abort_flag = 0;
-        for (int i = 0; i < kItemRing; ++i) {
-            mbar_init(smem_u32(&bars.item_full[i]), 1);
-            mbar_init(smem_u32(&bars.item_empty[i]), kItemReaders);
-        }
+        item_ring_init(bars.items, kItemReaders);
         mbar_init(smem_u32(&bars.q_full), 1);
         mbar_init(smem_u32(&bars.q_empty), 1);
         mbar_init(smem_u32(&bars.drain), 1);
@@ -265,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
             bool ok = true;
             for (uint32_t k = 0; ok; ++k) {
                 int w;
-                ok = claim_item(a, bars, k, w, wd);
+                ok = item_claim(bars.items, a.work, k, w, wd);
                 if (!ok || w >= a.n_items) break;
                 const Item it = decode_item(a, w);
                 if (q_iter > 0) ok = mbar_wait(smem_u32(&bars.q_empty), (q_iter - 1) & 1, wd);
@@ -315,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
             bool ok = true;
             for (uint32_t k = 0; ok; ++k) {
                 int w;
-                ok = read_item(bars, k, w, false, wd);
+                ok = item_read(bars.items, k, w, false, wd);
                 if (!ok || w >= a.n_items) break;
                 const Item it = decode_item(a, w);
                 KvIter kv(a, it);
@@ -394,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
         bool ok = true;
         for (uint32_t k = 0; ok; ++k) {
             int w;
-            ok = read_item(bars, k, w, true, wd);
+            ok = item_read(bars.items, k, w, true, wd);
             if (!ok || w >= a.n_items) break;
             const Item it = decode_item(a, w);
             float m = -INFINITY, l = 0.f;
