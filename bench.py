@@ -195,14 +195,18 @@ def oracle_sample(w, nrows_per_head, seed):
     return dt, flops, oracle.num_threads()
 
 
-def calibrate_rows(w, target_s, seed=0, lo=16, hi=4096):
+def calibrate_rows(w, target_s, seed=0, hi=4096):
     """Rows per head that make one oracle sample take about target_s seconds
-    (two-point fit: the per-call fixed cost is separated from the per-row cost)."""
+    (two-point fit: the per-call fixed cost is separated from the per-row cost).
+    Both fit points keep every oracle thread busy (the oracle hands rows out in
+    chunks of 4), else the per-row cost would come out too small."""
+    import oracle
+    lo = max(64, 8 * oracle.num_threads())
     t_lo, _, _ = oracle_sample(w, lo, seed)
     t_hi, _, _ = oracle_sample(w, 4 * lo, seed + 1)
     per_row = max((t_hi - t_lo) / (3 * lo), 1e-6)
     fixed = max(t_lo - lo * per_row, 0.0)
-    return int(max(lo, min(hi, (target_s - fixed) / per_row)))
+    return int(max(16, min(hi, (target_s - fixed) / per_row)))
 
 
 def cpu_baseline(w, target_s=15.0):

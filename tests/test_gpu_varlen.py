@@ -135,3 +135,31 @@ def test_varlen_workload_sampled_rows():
     rows = sample_rows(w.S, 256, w.seed + 1000, w.chunk)
     rows = np.unique(np.concatenate([rows, np.array(w.cu_seqlens[1:-1]), np.array(w.cu_seqlens[1:-1]) - 1]))
     _check(q, k, v, w.P, w.order, list(w.cu_seqlens), w.causal, rows=rows)
+
+
+@pytest.mark.parametrize("B,H,Hkv,D,causal", [(2, 4, 4, 64, True), (3, 2, 1, 128, False)])
+def test_varlen_batched_and_d64(B, H, Hkv, D, causal):
+    # every batch row uses the same documents; D = 64 takes the other tile shape
+    cu = [0, 200, 201, 700, 1024]
+    q, k, v = _qkv(B, H, Hkv, 1024, D, 1700 + B + D, torch.bfloat16)
+    _check(q, k, v, 4, "zigzag", cu, causal)
+
+
+def test_varlen_backward_d64_batched():
+    import ring_ulysses_sequence_b200 as rm
+    B, H, Hkv, S, D, P, order, cu = 2, 2, 1, 512, 64, 2, "contiguous", [0, 100, 356, 512]
+    qn, kn, vn = _qkv(B, H, Hkv, S, D, 1800, torch.bfloat16)
+    don = make_tensor((B, H, S, D), 1804, torch.bfloat16, 0.5)
+    q, k, v, do = (to_rank_major(t, P, order).cuda() for t in (qn, kn, vn, don))
+    table = rm.varlen_bounds(cu, S, True)
+    o, lse = rm.ring_attn_fwd(q, k, v, P, True, order, bounds=table)
+    dq, dk, dv = rm.ring_attn_bwd(q, k, v, o, lse, do, P, True, order, bounds=table)
+    torch.cuda.synchronize()
+    dq, dk, dv = (to_natural(t.cpu(), P, order) for t in (dq, dk, dv))
+    rdq, rdkv = oracle.attn_bwd(qn.float(), kn.float(), vn.float(), don.float(), True,
+                                cu_seqlens=cu)
+    for b in range(B):
+        for h in range(H):
+            assert_close(dq[b, h].numpy(), rdq[(b, h)], BF16_MAX_ABS, BF16_MEAN_ABS, f"dQ[{b},{h}]")
+        assert_close(dk[b, 0].numpy(), rdkv[(b, 0)][0], BF16_MAX_ABS, BF16_MEAN_ABS, f"dK[{b}]")
+        assert_close(dv[b, 0].numpy(), rdkv[(b, 0)][1], BF16_MAX_ABS, BF16_MEAN_ABS, f"dV[{b}]")

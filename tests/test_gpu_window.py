@@ -140,3 +140,18 @@ def test_window_workload_sampled_rows():
     q, k, v = make_inputs(w)
     rows = sample_rows(w.S, 256, w.seed + 1000, w.chunk)
     _check_fwd(q, k, v, w.P, w.order, w.window, rows=rows)
+
+
+@pytest.mark.parametrize("W", [1, 100, 257])
+def test_window_d64_forward_and_backward(W):
+    B, H, Hkv, S, D, P, order = 1, 4, 2, 1024, 64, 4, "zigzag"
+    q, k, v = _qkv(B, H, Hkv, S, D, 1900 + W, torch.bfloat16)
+    _check_fwd(q, k, v, P, order, W)
+    do = make_tensor((B, H, S, D), 1950 + W, torch.bfloat16, 0.5)
+    dq, dk, dv = gpu_grads(q, k, v, do, P, order, W)
+    rdq, rdkv = oracle.attn_bwd(q.float(), k.float(), v.float(), do.float(), True, window=W)
+    for h in range(H):
+        assert_close(dq[0, h].numpy(), rdq[(0, h)], BF16_MAX_ABS, BF16_MEAN_ABS, f"dQ[{h}]")
+    for g in range(Hkv):
+        assert_close(dk[0, g].numpy(), rdkv[(0, g)][0], BF16_MAX_ABS, BF16_MEAN_ABS, f"dK[{g}]")
+        assert_close(dv[0, g].numpy(), rdkv[(0, g)][1], BF16_MAX_ABS, BF16_MEAN_ABS, f"dV[{g}]")
