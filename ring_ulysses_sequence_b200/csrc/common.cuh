@@ -7,7 +7,6 @@
 #include <cuda.h>
 #include <stdint.h>
 
-#include "exp2_poly.h"
 
 namespace rm {
 
@@ -469,34 +468,6 @@ __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
     asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
-__device__ __forceinline__ float max3f(float a, float b, float c) {
-    float d;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-    return d;
-}
-
-// Software 2^x for two values on the FMA/ALU pipes (relieves the MUFU unit).
-// 2^x = 2^n * 2^f, n = round(x) obtained by adding 1.5 * 2^23 (the integer
-// lands in the low mantissa bits), f = x - n in [-1/2, 1/2], 2^f by the
-// minimax-relative polynomial of exp2_poly.h, and 2^n added to the exponent
-// field. Inputs below -125 (masked scores are -inf) are clamped so that the
-// result stays a normal number no larger than 2^-124.
-__device__ __forceinline__ void exp2_soft2(float x0, float x1, float& y0, float& y1) {
-    const uint64_t magic = pk2(12582912.0f, 12582912.0f);
-    const uint64_t x = pk2(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-    const uint64_t t = add2(x, magic);
-    const uint64_t f = sub2(x, sub2(t, magic));
-    uint64_t p = fma2(pk2(RM_EXP2_C4, RM_EXP2_C4), f, pk2(RM_EXP2_C3, RM_EXP2_C3));
-    p = fma2(p, f, pk2(RM_EXP2_C2, RM_EXP2_C2));
-    p = fma2(p, f, pk2(RM_EXP2_C1, RM_EXP2_C1));
-    p = fma2(p, f, pk2(RM_EXP2_C0, RM_EXP2_C0));
-    float p0, p1, t0, t1;
-    upk2(p, p0, p1);
-    upk2(t, t0, t1);
-    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);
