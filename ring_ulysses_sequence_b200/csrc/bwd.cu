@@ -21,6 +21,9 @@
 //                      tiles in ring order (i - t) mod P:
 //                        S = Q K^T, dP = dO V^T; dS -> bf16 in TMEM;
 //                        dQ += dS K
+//                      S has two TMEM buffers (the kernel leaves 128 columns
+//                      free), so S of tile j + 1 runs on the tensor pipe while
+//                      the compute warps turn tile j's S, dP into dS.
 // Warp roles as in the forward: warps 0-7 compute (two warpgroups splitting the
 // 128 columns of S), warp 8 issues UMMA, warp 9 issues TMA. TMEM (512 cols):
 // S [0,128), dP [128,256), accumulators at 256 and 384.
@@ -39,6 +42,8 @@ constexpr int kThreads = 320;
 constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;
 constexpr int kStages = 2;
+constexpr int kKRing = 3;        // dQ kernel: K tiles in flight (S runs a tile ahead of dQ)
+constexpr int kVRing = 2;        // dQ kernel: V tiles in flight
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
@@ -49,9 +54,10 @@ struct BCfg {
     // dK/dV kernel: K, V resident; stages of Q + dO + LSE + Delta
     static constexpr int kStageKV = 2 * kTile + 2 * kT * 4;
     static constexpr int kKvBarOff = 2 * kTile + kStages * kStageKV;
-    // dQ kernel: Q, dO resident; stages of K + V
-    static constexpr int kStageQ = 2 * kTile;
-    static constexpr int kQBarOff = 2 * kTile + kStages * kStageQ;
+    // dQ kernel: Q, dO resident; a ring of K tiles and a ring of V tiles
+    static constexpr int kKRingOff = 2 * kTile;
+    static constexpr int kVRingOff = kKRingOff + kKRing * kTile;
+    static constexpr int kQBarOff = kVRingOff + kVRing * kTile;
     static constexpr int kSmemKV = kKvBarOff + 256 + 1024;
     static constexpr int kSmemQ = kQBarOff + 256 + 1024;
 };
@@ -87,6 +93,17 @@ struct Bars {
     int abort_flag;
 };
 static_assert(sizeof(Bars) <= 256, "barrier block");
+
+// Barriers of the dQ kernel: separate rings for K and V tiles.
+struct QBars {
+    ItemRing items;
+    uint64_t res_full, res_empty, drain, acc_full;
+    uint64_t k_full[kKRing], k_empty[kKRing], v_full[kVRing], v_empty[kVRing];
+    uint64_t s_full, p_full;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+static_assert(sizeof(QBars) <= 256, "barrier block");
 
 // -------------------------------------------------------------------- dK / dV
 
@@ -484,10 +501,11 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
-    Bars& bars = *reinterpret_cast<Bars*>(smem + BCfg<D>::kQBarOff);
+    QBars& bars = *reinterpret_cast<QBars*>(smem + BCfg<D>::kQBarOff);
     const uint32_t q_smem = smem_u32(smem);
     const uint32_t do_smem = q_smem + BCfg<D>::kTile;
-    const uint32_t st_smem = q_smem + 2 * BCfg<D>::kTile;  // stage s: K, V
+    const uint32_t kr_smem = q_smem + BCfg<D>::kKRingOff;  // slot s: one K tile
+    const uint32_t vr_smem = q_smem + BCfg<D>::kVRingOff;  // slot s: one V tile
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -497,9 +515,13 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
         mbar_init(smem_u32(&bars.res_empty), 1);
         mbar_init(smem_u32(&bars.drain), 1);
         mbar_init(smem_u32(&bars.acc_full), 1);
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(smem_u32(&bars.st_full[s]), 1);
-            mbar_init(smem_u32(&bars.st_empty[s]), 1);
+        for (int s = 0; s < kKRing; ++s) {
+            mbar_init(smem_u32(&bars.k_full[s]), 1);
+            mbar_init(smem_u32(&bars.k_empty[s]), 1);
+        }
+        for (int s = 0; s < kVRing; ++s) {
+            mbar_init(smem_u32(&bars.v_full[s]), 1);
+            mbar_init(smem_u32(&bars.v_empty[s]), 1);
         }
         mbar_init(smem_u32(&bars.s_full), 1);
         mbar_init(smem_u32(&bars.p_full), 256);
@@ -521,8 +543,21 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
             prefetch_tmap(&a.tm_k);
             prefetch_tmap(&a.tm_v);
             prefetch_tmap(&a.tm_do);
-            uint32_t items = 0, fills = 0;
+            uint32_t items = 0, kf = 0, vf = 0;
             bool ok = true;
+            // one tile into slot (n % ring) of a ring, once its previous use is released
+            auto fill = [&](uint64_t* full, uint64_t* empty, int ring, uint32_t n, uint32_t dst,
+                            const CUtensorMap* map, int row) -> bool {
+                const int slot = n % ring;
+                if (n >= static_cast<uint32_t>(ring) &&
+                    !mbar_wait(smem_u32(&empty[slot]), (n / ring - 1) & 1, wd))
+                    return false;
+                mbar_arrive_expect_tx(smem_u32(&full[slot]), BCfg<D>::kTile);
+                for (int bx = 0; bx < BCfg<D>::kBoxes; ++bx)
+                    tma_load_2d(dst + slot * BCfg<D>::kTile + bx * BCfg<D>::kBox, map, bx * 64, row,
+                                smem_u32(&full[slot]));
+                return true;
+            };
             for (uint32_t k = 0; ok; ++k, ++items) {
                 int w;
                 ok = item_claim(bars.items, a.work, k, w, wd);
@@ -539,62 +574,81 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
                 KIter ki(a, it);
                 int kslot, cls;
                 while (ok && ki.next(a, kslot, cls)) {
-                    const int st = fills % kStages;
-                    const uint32_t use = fills / kStages;
-                    if (use > 0) ok = mbar_wait(smem_u32(&bars.st_empty[st]), (use - 1) & 1, wd);
-                    if (!ok) break;
-                    const uint32_t base = st_smem + st * BCfg<D>::kStageQ;
                     const int krow = (it.b * a.Hkv + it.g) * a.S + kslot;
-                    const uint32_t bar = smem_u32(&bars.st_full[st]);
-                    mbar_arrive_expect_tx(bar, BCfg<D>::kStageQ);
-                    for (int bx = 0; bx < BCfg<D>::kBoxes; ++bx) {
-                        tma_load_2d(base + bx * BCfg<D>::kBox, &a.tm_k, bx * 64, krow, bar);
-                        tma_load_2d(base + BCfg<D>::kTile + bx * BCfg<D>::kBox, &a.tm_v, bx * 64, krow, bar);
-                    }
-                    ++fills;
+                    ok = fill(bars.k_full, bars.k_empty, kKRing, kf, kr_smem, &a.tm_k, krow);
+                    if (!ok) break;
+                    ++kf;
+                    ok = fill(bars.v_full, bars.v_empty, kVRing, vf, vr_smem, &a.tm_v, krow);
+                    if (!ok) break;
+                    ++vf;
                 }
             }
             if (!ok) {
                 volatile int no_abort = 0;
                 const Watchdog w2{a.status, &no_abort, a.timeout_ns};
-                for (uint32_t i = fills > kStages ? fills - kStages : 0; i < fills; ++i)
-                    (void)mbar_wait(smem_u32(&bars.st_full[i % kStages]), (i / kStages) & 1, w2);
+                for (uint32_t i = kf > kKRing ? kf - kKRing : 0; i < kf; ++i)
+                    (void)mbar_wait(smem_u32(&bars.k_full[i % kKRing]), (i / kKRing) & 1, w2);
+                for (uint32_t i = vf > kVRing ? vf - kVRing : 0; i < vf; ++i)
+                    (void)mbar_wait(smem_u32(&bars.v_full[i % kVRing]), (i / kVRing) & 1, w2);
                 if (items > 0) (void)mbar_wait(smem_u32(&bars.res_full), (items - 1) & 1, w2);
             }
         }
     } else if (warp == kMmaWarp) {
         if (lane == 0) {
-            const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
-            uint32_t items = 0, uses = 0, p_cnt = 0;
+            const uint32_t tS[2] = {tmem, tmem + 128};
+            const uint32_t tdP = tmem + 256, tdQ = tmem + 384;
+            uint32_t items = 0, kc = 0, vc = 0, p_cnt = 0;
             bool ok = true;
             for (uint32_t k = 0; ok; ++k, ++items) {
                 int w;
                 ok = item_read(bars.items, k, w, false, wd);
                 if (!ok || w >= a.n_items) break;
                 const QItem it = decode_q_item(a, w);
-                KIter ki(a, it);
-                int ks, kc;
+                KIter ki(a, it);  // one tile ahead of the S products
+                int ks, kcls;
                 ok = mbar_wait(smem_u32(&bars.res_full), items & 1, wd);
                 if (!ok) break;
-                tc_fence_after();
-                for (int j = 0; ok && ki.next(a, ks, kc); ++j) {
-                    const int st = uses % kStages;
-                    ok = mbar_wait(smem_u32(&bars.st_full[st]), (uses / kStages) & 1, wd);
-                    if (!ok) break;
-                    ++uses;
+                const uint32_t bk = kc, bv = vc;
+                // S_j = Q K_j^T into buffer j & 1
+                auto score = [&](uint32_t j) -> bool {
+                    const uint32_t n = bk + j;
+                    if (!mbar_wait(smem_u32(&bars.k_full[n % kKRing]), (n / kKRing) & 1, wd)) return false;
                     tc_fence_after();
-                    const uint32_t k_addr = st_smem + st * BCfg<D>::kStageQ;
-                    const uint32_t v_addr = k_addr + BCfg<D>::kTile;
-                    issue_tile_product<D>(tS, q_smem, k_addr);     // S = Q K^T
-                    issue_tile_product<D>(tdP, do_smem, v_addr);   // dP = dO V^T
+                    issue_tile_product<D>(tS[j & 1], q_smem, kr_smem + (n % kKRing) * BCfg<D>::kTile);
+                    return true;
+                };
+                // dP_j = dO V_j^T; with it tile j is complete
+                auto dprod = [&](uint32_t j) -> bool {
+                    const uint32_t n = bv + j;
+                    if (!mbar_wait(smem_u32(&bars.v_full[n % kVRing]), (n / kVRing) & 1, wd)) return false;
+                    tc_fence_after();
+                    issue_tile_product<D>(tdP, do_smem, vr_smem + (n % kVRing) * BCfg<D>::kTile);
+                    umma_commit(smem_u32(&bars.v_empty[n % kVRing]));
                     umma_commit(smem_u32(&bars.s_full));
+                    return true;
+                };
+                (void)ki.next(a, ks, kcls);  // tile 0 (every query tile has one)
+                bool have1 = ki.next(a, ks, kcls);
+                ok = score(0) && dprod(0) && (!have1 || score(1));
+                uint32_t j = 0;
+                for (; ok; ++j) {
                     ok = mbar_wait(smem_u32(&bars.p_full), (p_cnt++) & 1, wd);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_acc_product<D>(tdQ, tdP, k_addr, j > 0);   // dQ += dS K
-                    umma_commit(smem_u32(&bars.st_empty[st]));
+                    const uint32_t n = bk + j;
+                    issue_acc_product<D>(tdQ, tdP, kr_smem + (n % kKRing) * BCfg<D>::kTile, j > 0);  // dQ += dS K
+                    umma_commit(smem_u32(&bars.k_empty[n % kKRing]));
+                    if (!have1) break;
+                    // dP of tile j + 1 overwrites dS_j after dQ has read it (in-order pipe)
+                    ok = dprod(j + 1);
+                    if (!ok) break;
+                    const bool have2 = ki.next(a, ks, kcls);
+                    if (have2) ok = score(j + 2);  // buffer j & 1: tile j's S has been read
+                    have1 = have2;
                 }
                 if (!ok) break;
+                kc = bk + j + 1;
+                vc = bv + j + 1;
                 umma_commit(smem_u32(&bars.acc_full));
                 umma_commit(smem_u32(&bars.res_empty));
             }
@@ -608,10 +662,10 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;      // query row of the tile = TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-        const uint32_t tS = tmem + lane_off + 64 * wg;
-        const uint32_t tdP = tmem + lane_off + 128 + 64 * wg;
+        const uint32_t tS0 = tmem + lane_off + 64 * wg;
+        const uint32_t tdP = tmem + lane_off + 256 + 64 * wg;
         constexpr int HC = D / 2;
-        const uint32_t tdQ = tmem + lane_off + 256 + HC * wg;
+        const uint32_t tdQ = tmem + lane_off + 384 + HC * wg;
         const float sl2 = a.scale_log2;
         uint32_t s_cnt = 0, items = 0;
         bool ok = true;
@@ -625,7 +679,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
             const float delta = a.delta[qrow];
             KIter ki(a, it);
             int kslot, cls;
-            while (ok && ki.next(a, kslot, cls)) {
+            for (uint32_t j = 0; ok && ki.next(a, kslot, cls); ++j) {
                 // query row r sees key column c iff lo(i) <= kpos + c <= hi(i)
                 int lo = 0;
                 unsigned wk = 0;
@@ -638,7 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
                 if (!ok) break;
                 tc_fence_after();
                 uint32_t sv[64], dpv[64];
-                tmem_ld64(tS, sv);
+                tmem_ld64(tS0 + 128 * (j & 1), sv);
                 tmem_ld64(tdP, dpv);
                 uint32_t dsk[32];
                 const uint64_t sl2x2 = pk2(sl2, sl2), nlse2 = pk2(-lse2, -lse2), del2 = pk2(delta, delta);
