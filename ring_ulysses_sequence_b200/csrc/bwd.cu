@@ -88,7 +88,7 @@ struct Bars {
     ItemRing items;  // work items claimed by the producer (dynamic distribution)
     uint64_t res_full, res_empty, drain, acc_full;
     uint64_t st_full[kStages], st_empty[kStages];
-    uint64_t s_full, p_full;
+    uint64_t s_full, p_half, p_full;  // S^T/dP^T in TMEM; P^T written; dS^T written
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -236,6 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
             mbar_init(smem_u32(&bars.st_empty[s]), 1);
         }
         mbar_init(smem_u32(&bars.s_full), 1);
+        mbar_init(smem_u32(&bars.p_half), 256);
         mbar_init(smem_u32(&bars.p_full), 256);
         fence_barrier_init();
     }
@@ -324,10 +325,14 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
                     issue_tile_product<D>(tS, k_smem, q_addr);     // S^T = K Q^T
                     issue_tile_product<D>(tdP, v_smem, do_addr);   // dP^T = V dO^T
                     umma_commit(smem_u32(&bars.s_full));
-                    ok = mbar_wait(smem_u32(&bars.p_full), (p_cnt++) & 1, wd);
+                    // dV runs while the compute warps work out dS^T
+                    ok = mbar_wait(smem_u32(&bars.p_half), p_cnt & 1, wd);
                     if (!ok) break;
                     tc_fence_after();
                     issue_acc_product<D>(tdV, tS, do_addr, j > 0);   // dV += P^T dO
+                    ok = mbar_wait(smem_u32(&bars.p_full), (p_cnt++) & 1, wd);
+                    if (!ok) break;
+                    tc_fence_after();
                     issue_acc_product<D>(tdK, tdP, q_addr, j > 0);   // dK += dS^T Q
                     umma_commit(smem_u32(&bars.st_empty[st]));
                 }
@@ -377,23 +382,24 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
                 ok = mbar_wait(smem_u32(&bars.s_full), (s_cnt++) & 1, wd);
                 if (!ok) break;
                 tc_fence_after();
-                // two quarters of 32 query columns: load S^T and dP^T, write
-                // bf16 P^T and dS^T over S^T/dP^T columns already read. LSE and
-                // Delta of the columns come four at a time from shared memory;
-                // the arithmetic runs on packed fp32 pairs.
+                // Two passes over two quarters of 32 query columns. Pass 1: P^T
+                // from S^T and LSE, written as bf16 over S^T columns already
+                // read (dV can start); pass 2: dS^T = P^T (dP^T - Delta) from the
+                // fp32 P kept in registers, written over dP^T. LSE and Delta come
+                // four at a time from shared memory; the arithmetic runs on
+                // packed fp32 pairs.
                 const uint64_t sl2x2 = pk2(sl2, sl2);
                 const uint64_t nlog2e = pk2(-kLog2e, -kLog2e);
+                uint64_t pp[32];  // P of this thread's 64 query columns, in pairs
 #pragma unroll
                 for (int qq = 0; qq < 2; ++qq) {
-                    uint32_t sv[32], dpv[32];
+                    uint32_t sv[32];
                     tmem_ld32(tS + 32 * qq, sv);
-                    tmem_ld32(tdP + 32 * qq, dpv);
                     const float4* lse4 = reinterpret_cast<const float4*>(lse_s + 64 * wg + 32 * qq);
-                    const float4* del4 = reinterpret_cast<const float4*>(del_s + 64 * wg + 32 * qq);
-                    uint32_t pk[16], dsk[16];
+                    uint32_t pk[16];
 #pragma unroll
                     for (int c4 = 0; c4 < 8; ++c4) {
-                        const float4 L = lse4[c4], Dl = del4[c4];
+                        const float4 L = lse4[c4];
 #pragma unroll
                         for (int hh = 0; hh < 2; ++hh) {
                             const int c = 4 * c4 + 2 * hh;
@@ -406,16 +412,35 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
                                 if (static_cast<unsigned>(q0 - lo) > wq) p0 = 0.f;
                                 if (static_cast<unsigned>(q0 + 1 - lo) > wq) p1 = 0.f;
                             }
-                            const uint64_t pp = pk2(p0, p1);
-                            const uint64_t dd = mul2(pp, sub2(pk2(__uint_as_float(dpv[c]), __uint_as_float(dpv[c + 1])),
-                                                              hh ? pk2(Dl.z, Dl.w) : pk2(Dl.x, Dl.y)));
-                            float d0, d1;
-                            upk2(dd, d0, d1);
+                            pp[16 * qq + (c >> 1)] = pk2(p0, p1);
                             pk[c >> 1] = pack_bf16x2(p0, p1);
-                            dsk[c >> 1] = pack_bf16x2(d0, d1);
                         }
                     }
                     tmem_st16(tS + 16 * qq, pk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(smem_u32(&bars.p_half));
+#pragma unroll
+                for (int qq = 0; qq < 2; ++qq) {
+                    uint32_t dpv[32];
+                    tmem_ld32(tdP + 32 * qq, dpv);
+                    const float4* del4 = reinterpret_cast<const float4*>(del_s + 64 * wg + 32 * qq);
+                    uint32_t dsk[16];
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        const float4 Dl = del4[c4];
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const int c = 4 * c4 + 2 * hh;
+                            const uint64_t dd = mul2(pp[16 * qq + (c >> 1)],
+                                                     sub2(pk2(__uint_as_float(dpv[c]), __uint_as_float(dpv[c + 1])),
+                                                          hh ? pk2(Dl.z, Dl.w) : pk2(Dl.x, Dl.y)));
+                            float d0, d1;
+                            upk2(dd, d0, d1);
+                            dsk[c >> 1] = pack_bf16x2(d0, d1);
+                        }
+                    }
                     tmem_st16(tdP + 16 * qq, dsk);
                 }
                 tmem_wait_st();
