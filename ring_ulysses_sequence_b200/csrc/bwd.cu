@@ -88,7 +88,8 @@ struct Bars {
     ItemRing items;  // work items claimed by the producer (dynamic distribution)
     uint64_t res_full, res_empty, drain, acc_full;
     uint64_t st_full[kStages], st_empty[kStages];
-    uint64_t s_full, p_half, p_full;  // S^T/dP^T in TMEM; P^T written; dS^T written
+    uint64_t s_full, dp_full;         // S^T in TMEM; dP^T in TMEM
+    uint64_t p_half, p_full;          // P^T written; dS^T written
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -99,7 +100,9 @@ struct QBars {
     ItemRing items;
     uint64_t res_full, res_empty, drain, acc_full;
     uint64_t k_full[kKRing], k_empty[kKRing], v_full[kVRing], v_empty[kVRing];
-    uint64_t s_full, p_full;
+    uint64_t s_full[2];   // S of buffer b is in TMEM (S runs up to two tiles ahead)
+    uint64_t dp_full;     // dP of the next tile is in TMEM
+    uint64_t p_full;      // dS written
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -236,6 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
             mbar_init(smem_u32(&bars.st_empty[s]), 1);
         }
         mbar_init(smem_u32(&bars.s_full), 1);
+        mbar_init(smem_u32(&bars.dp_full), 1);
         mbar_init(smem_u32(&bars.p_half), 256);
         mbar_init(smem_u32(&bars.p_full), 256);
         fence_barrier_init();
@@ -323,8 +327,9 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
                     const uint32_t q_addr = st_smem + st * BCfg<D>::kStageKV;
                     const uint32_t do_addr = q_addr + BCfg<D>::kTile;
                     issue_tile_product<D>(tS, k_smem, q_addr);     // S^T = K Q^T
+                    umma_commit(smem_u32(&bars.s_full));           // P^T can start
                     issue_tile_product<D>(tdP, v_smem, do_addr);   // dP^T = V dO^T
-                    umma_commit(smem_u32(&bars.s_full));
+                    umma_commit(smem_u32(&bars.dp_full));
                     // dV runs while the compute warps work out dS^T
                     ok = mbar_wait(smem_u32(&bars.p_half), p_cnt & 1, wd);
                     if (!ok) break;
@@ -356,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
         const uint32_t tdV = tmem + lane_off + 256 + HC * wg;
         const uint32_t tdK = tmem + lane_off + 384 + HC * wg;
         const float sl2 = a.scale_log2;
-        uint32_t uses = 0, s_cnt = 0, items = 0;
+        uint32_t uses = 0, s_cnt = 0, items = 0;  // s_cnt counts tiles for s_full and dp_full
         bool ok = true;
         for (uint32_t k = 0; ok; ++k, ++items) {
             int w;
@@ -379,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
                 const float* lse_s = reinterpret_cast<const float*>(
                     smem + 2 * BCfg<D>::kTile + st * BCfg<D>::kStageKV + 2 * BCfg<D>::kTile);
                 const float* del_s = lse_s + kT;
-                ok = mbar_wait(smem_u32(&bars.s_full), (s_cnt++) & 1, wd);
+                ok = mbar_wait(smem_u32(&bars.s_full), s_cnt & 1, wd);
                 if (!ok) break;
                 tc_fence_after();
                 // Two passes over two quarters of 32 query columns. Pass 1: P^T
@@ -421,6 +426,9 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(smem_u32(&bars.p_half));
+                ok = mbar_wait(smem_u32(&bars.dp_full), (s_cnt++) & 1, wd);
+                if (!ok) break;
+                tc_fence_after();
 #pragma unroll
                 for (int qq = 0; qq < 2; ++qq) {
                     uint32_t dpv[32];
@@ -548,7 +556,9 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
             mbar_init(smem_u32(&bars.v_full[s]), 1);
             mbar_init(smem_u32(&bars.v_empty[s]), 1);
         }
-        mbar_init(smem_u32(&bars.s_full), 1);
+        mbar_init(smem_u32(&bars.s_full[0]), 1);
+        mbar_init(smem_u32(&bars.s_full[1]), 1);
+        mbar_init(smem_u32(&bars.dp_full), 1);
         mbar_init(smem_u32(&bars.p_full), 256);
         fence_barrier_init();
     }
@@ -640,16 +650,17 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
                     if (!mbar_wait(smem_u32(&bars.k_full[n % kKRing]), (n / kKRing) & 1, wd)) return false;
                     tc_fence_after();
                     issue_tile_product<D>(tS[j & 1], q_smem, kr_smem + (n % kKRing) * BCfg<D>::kTile);
+                    umma_commit(smem_u32(&bars.s_full[j & 1]));
                     return true;
                 };
-                // dP_j = dO V_j^T; with it tile j is complete
+                // dP_j = dO V_j^T
                 auto dprod = [&](uint32_t j) -> bool {
                     const uint32_t n = bv + j;
                     if (!mbar_wait(smem_u32(&bars.v_full[n % kVRing]), (n / kVRing) & 1, wd)) return false;
                     tc_fence_after();
                     issue_tile_product<D>(tdP, do_smem, vr_smem + (n % kVRing) * BCfg<D>::kTile);
                     umma_commit(smem_u32(&bars.v_empty[n % kVRing]));
-                    umma_commit(smem_u32(&bars.s_full));
+                    umma_commit(smem_u32(&bars.dp_full));
                     return true;
                 };
                 (void)ki.next(a, ks, kcls);  // tile 0 (every query tile has one)
@@ -692,7 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
         constexpr int HC = D / 2;
         const uint32_t tdQ = tmem + lane_off + 384 + HC * wg;
         const float sl2 = a.scale_log2;
-        uint32_t s_cnt = 0, items = 0;
+        uint32_t s_cnt[2] = {0, 0}, dp_cnt = 0, items = 0;
         bool ok = true;
         for (uint32_t k = 0; ok; ++k, ++items) {
             int w;
@@ -713,29 +724,47 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
                     lo = rb.x - ki.kpos;
                     wk = static_cast<unsigned>(rb.y - rb.x);
                 }
-                ok = mbar_wait(smem_u32(&bars.s_full), (s_cnt++) & 1, wd);
+                // P from S as soon as S is in (it may be a tile ahead of dP)
+                const int b = j & 1;
+                ok = mbar_wait(smem_u32(&bars.s_full[b]), (s_cnt[b]++) & 1, wd);
                 if (!ok) break;
                 tc_fence_after();
-                uint32_t sv[64], dpv[64];
-                tmem_ld64(tS0 + 128 * (j & 1), sv);
-                tmem_ld64(tdP, dpv);
-                uint32_t dsk[32];
-                const uint64_t sl2x2 = pk2(sl2, sl2), nlse2 = pk2(-lse2, -lse2), del2 = pk2(delta, delta);
+                uint64_t pp[32];
+                {
+                    uint32_t sv[64];
+                    tmem_ld64(tS0 + 128 * b, sv);
+                    const uint64_t sl2x2 = pk2(sl2, sl2), nlse2 = pk2(-lse2, -lse2);
 #pragma unroll
-                for (int c = 0; c < 64; c += 2) {
-                    const int k0 = 64 * wg + c;
-                    float x0, x1;
-                    upk2(fma2(pk2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, nlse2), x0, x1);
-                    float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                    if (cls == kMask) {
-                        if (static_cast<unsigned>(k0 - lo) > wk) p0 = 0.f;
-                        if (static_cast<unsigned>(k0 + 1 - lo) > wk) p1 = 0.f;
+                    for (int c = 0; c < 64; c += 2) {
+                        const int k0 = 64 * wg + c;
+                        float x0, x1;
+                        upk2(fma2(pk2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, nlse2), x0, x1);
+                        float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                        if (cls == kMask) {
+                            if (static_cast<unsigned>(k0 - lo) > wk) p0 = 0.f;
+                            if (static_cast<unsigned>(k0 + 1 - lo) > wk) p1 = 0.f;
+                        }
+                        pp[c >> 1] = pk2(p0, p1);
                     }
-                    float d0, d1;
-                    upk2(mul2(pk2(p0, p1), sub2(pk2(__uint_as_float(dpv[c]), __uint_as_float(dpv[c + 1])), del2)), d0, d1);
-                    dsk[c >> 1] = pack_bf16x2(d0, d1);
                 }
-                tmem_st32(tdP, dsk);
+                // then dS = P (dP - Delta), written over dP
+                ok = mbar_wait(smem_u32(&bars.dp_full), (dp_cnt++) & 1, wd);
+                if (!ok) break;
+                tc_fence_after();
+                const uint64_t del2 = pk2(delta, delta);
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    uint32_t dpv[32], dsk[16];
+                    tmem_ld32(tdP + 32 * h2, dpv);
+#pragma unroll
+                    for (int c = 0; c < 32; c += 2) {
+                        float d0, d1;
+                        upk2(mul2(pp[16 * h2 + (c >> 1)],
+                                  sub2(pk2(__uint_as_float(dpv[c]), __uint_as_float(dpv[c + 1])), del2)), d0, d1);
+                        dsk[c >> 1] = pack_bf16x2(d0, d1);
+                    }
+                    tmem_st16(tdP + 16 * h2, dsk);
+                }
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(smem_u32(&bars.p_full));
