@@ -318,28 +318,52 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
                 ok = mbar_wait(smem_u32(&bars.res_full), items & 1, wd);
                 if (!ok) break;
                 tc_fence_after();
-                for (int j = 0; ok && qi.next(a, qh, qs, qc); ++j) {
-                    const int st = uses % kStages;
-                    ok = mbar_wait(smem_u32(&bars.st_full[st]), (uses / kStages) & 1, wd);
-                    if (!ok) break;
+                // S^T of query tile j + 1 is issued right after dV of tile j (it
+                // overwrites P^T, which dV has read: in-order pipe), so the next
+                // tile's P^T pass runs while dK and dP^T finish on the tensor pipe.
+                auto stage = [&](int& st) -> bool {
+                    st = uses % kStages;
+                    const bool r = mbar_wait(smem_u32(&bars.st_full[st]), (uses / kStages) & 1, wd);
                     ++uses;
                     tc_fence_after();
+                    return r;
+                };
+                int st = 0;
+                (void)qi.next(a, qh, qs, qc);  // query tile 0 (every key tile has one)
+                ok = stage(st);
+                if (ok) {
+                    const uint32_t q_addr = st_smem + st * BCfg<D>::kStageKV;
+                    issue_tile_product<D>(tS, k_smem, q_addr);                     // S^T = K Q^T
+                    umma_commit(smem_u32(&bars.s_full));
+                    issue_tile_product<D>(tdP, v_smem, q_addr + BCfg<D>::kTile);   // dP^T = V dO^T
+                    umma_commit(smem_u32(&bars.dp_full));
+                }
+                for (int j = 0; ok; ++j) {
                     const uint32_t q_addr = st_smem + st * BCfg<D>::kStageKV;
                     const uint32_t do_addr = q_addr + BCfg<D>::kTile;
-                    issue_tile_product<D>(tS, k_smem, q_addr);     // S^T = K Q^T
-                    umma_commit(smem_u32(&bars.s_full));           // P^T can start
-                    issue_tile_product<D>(tdP, v_smem, do_addr);   // dP^T = V dO^T
-                    umma_commit(smem_u32(&bars.dp_full));
                     // dV runs while the compute warps work out dS^T
                     ok = mbar_wait(smem_u32(&bars.p_half), p_cnt & 1, wd);
                     if (!ok) break;
                     tc_fence_after();
                     issue_acc_product<D>(tdV, tS, do_addr, j > 0);   // dV += P^T dO
+                    const bool have_next = qi.next(a, qh, qs, qc);
+                    int st_next = st;
+                    if (have_next) {
+                        ok = stage(st_next);
+                        if (!ok) break;
+                        issue_tile_product<D>(tS, k_smem, st_smem + st_next * BCfg<D>::kStageKV);
+                        umma_commit(smem_u32(&bars.s_full));
+                    }
                     ok = mbar_wait(smem_u32(&bars.p_full), (p_cnt++) & 1, wd);
                     if (!ok) break;
                     tc_fence_after();
                     issue_acc_product<D>(tdK, tdP, q_addr, j > 0);   // dK += dS^T Q
                     umma_commit(smem_u32(&bars.st_empty[st]));
+                    if (!have_next) break;
+                    // dP^T of the next tile overwrites dS^T after dK has read it
+                    issue_tile_product<D>(tdP, v_smem, st_smem + st_next * BCfg<D>::kStageKV + BCfg<D>::kTile);
+                    umma_commit(smem_u32(&bars.dp_full));
+                    st = st_next;
                 }
                 if (!ok) break;
                 umma_commit(smem_u32(&bars.acc_full));
