@@ -174,3 +174,15 @@ def test_layout_validation(lib):
 def test_valid_call_without_gpu_reports_cuda_error(lib):
     assert fwd(lib) == 3
     assert lib.rm_last_cuda_error() != 0
+
+
+def test_binding_argument_counts_match_the_header():
+    # every RM_API declaration's parameter count equals the ctypes binding's
+    from ring_ulysses_sequence_b200 import native
+    text = open(HEADER).read()
+    decls = re.findall(r"^RM_API\s+[\w\s\*]*?\b(rm_\w+)\s*\(([^;]*?)\)\s*;", text, flags=re.M | re.S)
+    assert decls
+    for name, params in decls:
+        params = " ".join(params.split())
+        n = 0 if params in ("", "void") else params.count(",") + 1
+        assert len(native.SIGNATURES[name][1]) == n, (name, n, len(native.SIGNATURES[name][1]))
