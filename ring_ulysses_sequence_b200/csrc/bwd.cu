@@ -26,7 +26,11 @@
 //                      the compute warps turn tile j's S, dP into dS.
 // Warp roles as in the forward: warps 0-7 compute (two warpgroups splitting the
 // 128 columns of S), warp 8 issues UMMA, warp 9 issues TMA. TMEM (512 cols):
-// S [0,128), dP [128,256), accumulators at 256 and 384.
+// dK/dV: S^T [0,128), dP^T [128,256), dV at 256, dK at 384; dQ: S in two
+// buffers [0,128) and [128,256), dP [256,384), dQ at 384. The elementwise step
+// runs in two passes, P first (the MMA thread can start the product that needs
+// only P) and dS second, and S and dP signal separately, so the compute warps
+// start P while dP is still on the tensor pipe.
 #include <algorithm>
 
 #include "common.cuh"
