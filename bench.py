@@ -43,7 +43,8 @@ def parse_args():
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--only", choices=["all", "fwd", "permute", "bwd", "window", "packed"],
+    p.add_argument("--only", choices=["all", "fwd", "permute", "bwd", "window", "packed",
+                                      "layout"],
                    default="all",
                    help="restrict to one kernel (used for profiling runs)")
     p.add_argument("--skip-cpu", action="store_true", help="skip the CPU oracle baseline")
@@ -390,6 +391,38 @@ def bench_permute(args, dev, stream):
             "gbs": moved / ms / 1e6, "launches": steps + max(3, args.warmup)}
 
 
+def bench_layout(args, dev, stream):
+    """The HBM-bound helpers on the bench workload's tensors: natural -> rank-major
+    reorder of Q (bf16), and the standalone (O, LSE) merge of one fp32 partial
+    into a running pair for every query row."""
+    import torch
+    import ring_ulysses_sequence_b200 as rm
+    from ring_ulysses_sequence_b200.synth import WORKLOADS, BENCH_WORKLOAD
+    w = WORKLOADS[BENCH_WORKLOAD]
+    q = torch.randn((w.B, w.H, w.S, w.D), device=dev).to(w.dtype)
+    q_rm = torch.empty_like(q)
+    rows = w.B * w.H * w.S
+    o_acc = torch.randn((rows, w.D), device=dev)
+    o_part = torch.randn((rows, w.D), device=dev)
+    l_acc = torch.randn(rows, device=dev)
+    l_part = torch.randn(rows, device=dev)
+    steps = max(5, min(args.steps, 50))
+    out = {}
+    for name, fn, moved in (
+            ("seq_reorder", lambda: rm.seq_reorder(q, w.P, w.order, "to_rank_major", out=q_rm,
+                                                   stream=stream),
+             2 * q.numel() * q.element_size()),
+            ("lse_merge", lambda: rm.lse_merge_(o_acc, l_acc, o_part, l_part, stream=stream),
+             (3 * rows * w.D + 3 * rows) * 4)):
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                fn()
+        torch.cuda.synchronize()
+        ms = time_on_stream(fn, steps, stream) / steps
+        out[name] = {"ms": ms, "bytes_per_launch": moved, "gbs": moved / ms / 1e6}
+    return out
+
+
 def bench_masked(args, dev, stream, name):
     """Forward with a sparser mask: the 32k GQA layer with a 4096-key causal
     window, or over packed documents."""
@@ -478,6 +511,8 @@ def main():
             out["fwd"] = bench_forward(w, args, dev, stream)
         if rank == 0 and args.only in ("all", "permute"):
             out["permute"] = bench_permute(args, dev, stream)
+        if rank == 0 and args.only in ("all", "layout"):
+            out["layout"] = bench_layout(args, dev, stream)
         if rank == 0 and args.only in ("all", "window"):
             out["window"] = bench_masked(args, dev, stream,
                                          "ring_fwd_bf16_S32k_gqa_causal_zigzag_window4k")
@@ -544,6 +579,14 @@ def main():
                          "unit": "GB/s", "frac": p["gbs"] / peaks["hbm_gbs"],
                          "peak_source": f"{peak_src} hbm_gbs",
                          "bytes_per_launch": p["bytes_per_launch"]}}
+    if "layout" in out:
+        for name, x in out["layout"].items():
+            extra[name] = {
+                "workload": f"{w.name} tensors", "ms": x["ms"], "GB/s": x["gbs"],
+                "roofline": {"bound": "hbm", "achieved": x["gbs"], "peak": peaks["hbm_gbs"],
+                             "unit": "GB/s", "frac": x["gbs"] / peaks["hbm_gbs"],
+                             "peak_source": f"{peak_src} hbm_gbs",
+                             "bytes_per_launch": x["bytes_per_launch"]}}
     for key, label in (("window", "ring_attn_fwd_window"), ("packed", "ring_attn_fwd_varlen")):
         if key not in out:
             continue
