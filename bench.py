@@ -44,7 +44,7 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--only", choices=["all", "fwd", "permute", "bwd", "window", "packed",
-                                      "layout"],
+                                      "layout", "allgather"],
                    default="all",
                    help="restrict to one kernel (used for profiling runs)")
     p.add_argument("--skip-cpu", action="store_true", help="skip the CPU oracle baseline")
@@ -423,6 +423,50 @@ def bench_layout(args, dev, stream):
     return out
 
 
+def bench_allgather(args, dev, stream):
+    """The all-gather alternative to the ring on the bench workload: gather K/V
+    into natural order (two reorders, the one-device form of the collective),
+    then one attention pass. Timed whole and attention alone; the per-rank K/V
+    residency of both designs in a real P-rank run is reported beside it."""
+    import torch
+    import ring_ulysses_sequence_b200 as rm
+    from ring_ulysses_sequence_b200.synth import WORKLOADS, BENCH_WORKLOAD
+    w = WORKLOADS[BENCH_WORKLOAD]
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed)
+    q, k, v = ((torch.randn(s, generator=g, device=dev) * w.input_scale).to(w.dtype)
+               for s in [(w.B, w.H, w.S, w.D), (w.B, w.Hkv, w.S, w.D), (w.B, w.Hkv, w.S, w.D)])
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.S), dtype=torch.float32, device=dev)
+    kv_all = [torch.empty_like(k), torch.empty_like(v)]
+
+    def gather():
+        rm.allgather_kv(k, v, w.P, w.order, outs=kv_all, stream=stream)
+
+    def attend():
+        rm.allgather_attn_fwd(q, kv_all[0], kv_all[1], w.P, w.causal, w.order, out=o, lse=lse,
+                              stream=stream)
+
+    def step():
+        gather()
+        attend()
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+    torch.cuda.synchronize()
+    steps = max(5, min(args.steps, 100))
+    ms = time_on_stream(step, steps, stream) / steps
+    ms_attn = time_on_stream(attend, steps, stream) / steps
+    if rm.native.rm_check_device_status(stream) != 0:
+        raise RuntimeError("device watchdog fired during the all-gather benchmark")
+    kv_block = 2 * (w.S // w.P) * w.B * w.Hkv * w.D * k.element_size()  # K + V of one rank
+    return {"workload": w.name, "ms_per_step": ms, "ms_attention": ms_attn,
+            "tflops": w.fwd_flops() / ms / 1e9, "tflops_attention": w.fwd_flops() / ms_attn / 1e9,
+            "flops_per_launch": w.fwd_flops(),
+            "kv_bytes_per_rank": {"ring": 2 * kv_block, "allgather": w.P * kv_block}}
+
+
 def bench_masked(args, dev, stream, name):
     """Forward with a sparser mask: the 32k GQA layer with a 4096-key causal
     window, or over packed documents."""
@@ -513,6 +557,8 @@ def main():
             out["permute"] = bench_permute(args, dev, stream)
         if rank == 0 and args.only in ("all", "layout"):
             out["layout"] = bench_layout(args, dev, stream)
+        if rank == 0 and args.only in ("all", "allgather"):
+            out["allgather"] = bench_allgather(args, dev, stream)
         if rank == 0 and args.only in ("all", "window"):
             out["window"] = bench_masked(args, dev, stream,
                                          "ring_fwd_bf16_S32k_gqa_causal_zigzag_window4k")
@@ -587,6 +633,18 @@ def main():
                              "unit": "GB/s", "frac": x["gbs"] / peaks["hbm_gbs"],
                              "peak_source": f"{peak_src} hbm_gbs",
                              "bytes_per_launch": x["bytes_per_launch"]}}
+    if "allgather" in out:
+        x = out["allgather"]
+        extra["allgather_attn_fwd"] = {
+            "workload": x["workload"], "ms_per_step": x["ms_per_step"], "TFLOPS": x["tflops"],
+            "ms_attention_only": x["ms_attention"], "TFLOPS_attention_only": x["tflops_attention"],
+            "step": "allgather_kv (K, V rank-major -> natural) + rm_allgather_attn_fwd",
+            "kv_bytes_resident_per_rank": x["kv_bytes_per_rank"],
+            "roofline": {"bound": "tensor", "achieved": x["tflops_attention"],
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": x["tflops_attention"] / peaks["bf16_tflops"],
+                         "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)",
+                         "flops_per_launch": x["flops_per_launch"]}}
     for key, label in (("window", "ring_attn_fwd_window"), ("packed", "ring_attn_fwd_varlen")):
         if key not in out:
             continue

@@ -98,6 +98,32 @@ RM_API rm_status rm_ring_attn_fwd(const void* q, const void* k, const void* v, v
                            rm_order order, rm_dtype dtype, float scale, cudaStream_t stream);
 
 /*
+ * rm_allgather_attn_fwd — the all-gather alternative to the ring (forward).
+ *
+ * The axolotl-ringmaster README (Benchmark section) offers two ways to bring
+ * every rank's keys to its queries: the p2p ring (O(S/P) keys resident per
+ * rank) and an "allgather" rotater that collects all keys first (faster, more
+ * memory). This is the second: each rank's queries attend, in one pass in
+ * position order, to the keys of all ranks gathered into natural token order.
+ * The result is the same attention as rm_ring_attn_fwd (up to fp32 rounding
+ * order).
+ *
+ *   q            [B, H,   S, D]  BF16, rank-major S (each rank's shard, as for
+ *                                the ring)
+ *   k_all, v_all [B, Hkv, S, D]  BF16, NATURAL token order: the gathered keys
+ *                                (rm_seq_reorder RANK_MAJOR_TO_NATURAL of the
+ *                                rank-major k and v forms them on one device)
+ *   o, lse       as rm_ring_attn_fwd (rank-major S)
+ *   P, order     the layout of q, o and lse.
+ *
+ * Shapes and validation as rm_ring_attn_fwd. FP32 returns RM_ERR_UNSUPPORTED.
+ */
+RM_API rm_status rm_allgather_attn_fwd(const void* q, const void* k_all, const void* v_all,
+                                       void* o, float* lse, int B, int H, int Hkv, int S, int D,
+                                       int P, int causal, rm_order order, rm_dtype dtype,
+                                       float scale, cudaStream_t stream);
+
+/*
  * rm_ring_attn_fwd_window — rm_ring_attn_fwd with a causal sliding window.
  *
  * The axolotl-ringmaster README's Status table (phase 4) lists sliding-window

@@ -85,6 +85,36 @@ def ring_attn_fwd(q, k, v, P, causal=True, order="zigzag", scale=None, out=None,
     return out, lse
 
 
+def allgather_kv(k, v, P, order="zigzag", outs=None, stream=None):
+    """The all-gather of the rank-major k, v [B,Hkv,S,D] on one device: both in
+    natural token order, for allgather_attn_fwd."""
+    k_all = seq_reorder(k, P, order, "to_natural", out=None if outs is None else outs[0],
+                        stream=stream)
+    v_all = seq_reorder(v, P, order, "to_natural", out=None if outs is None else outs[1],
+                        stream=stream)
+    return k_all, v_all
+
+
+def allgather_attn_fwd(q, k_all, v_all, P, causal=True, order="zigzag", scale=None, out=None,
+                       lse=None, stream=None):
+    """All-gather attention forward: q [B,H,S,D] rank-major, k_all/v_all
+    [B,Hkv,S,D] in natural order (allgather_kv). Returns rank-major (O, LSE),
+    the same attention as ring_attn_fwd."""
+    import torch
+    for t, n in ((q, "q"), (k_all, "k_all"), (v_all, "v_all")):
+        _need(t, n)
+    B, H, S, D = q.shape
+    Hkv = k_all.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    native.rm_allgather_attn_fwd(q, k_all, v_all, out, lse, B, H, Hkv, S, D, P, causal,
+                                 _order(order), _dtype_code(q), scale, stream)
+    return out, lse
+
+
 def ring_attn_bwd(q, k, v, o, lse, dout, P, causal=True, order="zigzag", scale=None,
                   workspace=None, stream=None, window=0, bounds=None):
     """Ring attention backward. Returns fp32 (dQ, dK, dV).

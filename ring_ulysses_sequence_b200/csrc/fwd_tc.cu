@@ -27,6 +27,12 @@
 // so the tensor pipe runs one tile's products while the other tile's softmax
 // runs. O is rescaled only when a row maximum grows by more than 2^8 (in exp2
 // units); the sum l uses the same reference maximum, so the result is exact.
+//
+// The all-gather variant (kGathered; the "allgather" rotater of the
+// axolotl-ringmaster README, Benchmark section: faster, more memory) runs the
+// same kernel with K/V already gathered from every rank into natural token
+// order: each query tile makes one pass over the visible key tiles in
+// position order instead of P ring steps.
 #include <algorithm>
 
 #include "common.cuh"
@@ -112,6 +118,10 @@ __device__ __forceinline__ Item decode_item(const TcArgs& a, int w) {
 // the tiles to visit in each run are an interval too: O(1) work per tile
 // returned, no division. kpos holds the natural position of the tile last
 // returned.
+//
+// Gathered variant: the keys are one run of all S positions in natural order
+// (slot = position), visited once.
+template <bool kGathered>
 struct KvIter {
     int rank, lo, hi, t, run, u, u_end, s0, p0, kpos;
     __device__ __forceinline__ KvIter(const TcArgs& a, const Item& it)
@@ -122,24 +132,38 @@ struct KvIter {
     // `a` is the kernel's parameter block itself
     __device__ __forceinline__ bool next(const TcArgs& a, int& kslot) {
         const RingLayout& lay = a.lay;
-        while (u >= u_end) {
-            const int runs = lay.zigzag ? 2 : 1;
-            if (++run == runs) {  // run starts at -1, so the first call opens run 0 of step 0
+        if constexpr (kGathered) {
+            if (u >= u_end) {
+                if (run >= 0) return false;  // run starts at -1: one run only
                 run = 0;
-                if (++t == lay.P) return false;
+                s0 = p0 = 0;
+                u = max(0, ceil_div128(lo - (kBN - 1)));
+                u_end = min(lay.S / kBN, max((hi >> 7) + 1, 0));
+                if (u >= u_end) return false;
             }
-            const int r = lay.owner(rank, t);
-            const int ctiles = (lay.zigzag ? lay.c : lay.L) / kBN;
-            s0 = r * lay.L + run * lay.c;
-            p0 = lay.zigzag ? (run == 0 ? r * lay.c : (2 * lay.P - 1 - r) * lay.c) : r * lay.L;
-            // tiles whose keys meet [lo, hi]: p0 + 128 u <= hi and p0 + 128 u + 127 >= lo
-            u = max(0, ceil_div128(lo - (kBN - 1) - p0));
-            u_end = min(ctiles, max(((hi - p0) >> 7) + 1, 0));
+            kpos = kslot = u * kBN;
+            ++u;
+            return true;
+        } else {
+            while (u >= u_end) {
+                const int runs = lay.zigzag ? 2 : 1;
+                if (++run == runs) {  // run starts at -1, so the first call opens run 0 of step 0
+                    run = 0;
+                    if (++t == lay.P) return false;
+                }
+                const int r = lay.owner(rank, t);
+                const int ctiles = (lay.zigzag ? lay.c : lay.L) / kBN;
+                s0 = r * lay.L + run * lay.c;
+                p0 = lay.zigzag ? (run == 0 ? r * lay.c : (2 * lay.P - 1 - r) * lay.c) : r * lay.L;
+                // tiles whose keys meet [lo, hi]: p0 + 128 u <= hi and p0 + 128 u + 127 >= lo
+                u = max(0, ceil_div128(lo - (kBN - 1) - p0));
+                u_end = min(ctiles, max(((hi - p0) >> 7) + 1, 0));
+            }
+            kpos = p0 + u * kBN;
+            kslot = s0 + u * kBN;
+            ++u;
+            return true;
         }
-        kpos = p0 + u * kBN;
-        kslot = s0 + u * kBN;
-        ++u;
-        return true;
     }
 };
 
@@ -177,7 +201,7 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint3
                 (accumulate || k > 0) ? 1u : 0u);
 }
 
-template <int D>
+template <int D, bool kGathered>
 __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_constant__ TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -237,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
                         tma_load_2d(q_smem + x * Cfg<D>::kTileBytes + bx * Cfg<D>::kBoxBytes, &a.tm_q,
                                     bx * 64, row, smem_u32(&bars.q_full));
                 }
-                KvIter kv(a, it);
+                KvIter<kGathered> kv(a, it);
                 int kslot;
                 while (ok && kv.next(a, kslot)) {
                     const int row = (it.b * a.Hkv + it.g) * a.S + kslot;
@@ -277,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
                 ok = item_read(bars.items, k, w, false, wd);
                 if (!ok || w >= a.n_items) break;
                 const Item it = decode_item(a, w);
-                KvIter kv(a, it);
+                KvIter<kGathered> kv(a, it);
                 int ks;
                 bool have_cur = kv.next(a, ks);   // tile 0 (every item has one)
                 bool have_next = kv.next(a, ks);  // tile 1
@@ -357,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
             if (!ok || w >= a.n_items) break;
             const Item it = decode_item(a, w);
             float m = -INFINITY, l = 0.f;
-            KvIter kv(a, it);
+            KvIter<kGathered> kv(a, it);
             const int qpos = x ? it.pos1 : it.pos0;
             const int2 bf = row_bounds(a.mk, qpos), bl = row_bounds(a.mk, qpos + kBM - 1);
             int kslot, j = 0;
@@ -472,6 +496,16 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
     }
 }
 
+template <int D, bool kGathered>
+cudaError_t launch(const TcArgs& a, int grid, const LaunchCtx& ctx) {
+    constexpr int smem = Cfg<D>::kSmemBytes;
+    cudaError_t e = cudaFuncSetAttribute(ring_fwd_tc_kernel<D, kGathered>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    ring_fwd_tc_kernel<D, kGathered><<<grid, kThreads, smem, ctx.stream>>>(a);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_fwd_tc(const AttnShape& sh, const void* q, const void* k, const void* v,
@@ -504,20 +538,9 @@ cudaError_t launch_fwd_tc(const AttnShape& sh, const void* q, const void* k, con
     a.lay = RingLayout{sh.S, sh.P, sh.S / sh.P, sh.zigzag ? sh.S / (2 * sh.P) : sh.S / sh.P,
                        sh.zigzag};
     const int grid = std::min(a.n_items, ctx.num_sms);
-    if (sh.D == 64) {
-        constexpr int smem = Cfg<64>::kSmemBytes;
-        if ((e = cudaFuncSetAttribute(ring_fwd_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      smem)) != cudaSuccess)
-            return e;
-        ring_fwd_tc_kernel<64><<<grid, kThreads, smem, ctx.stream>>>(a);
-    } else {
-        constexpr int smem = Cfg<128>::kSmemBytes;
-        if ((e = cudaFuncSetAttribute(ring_fwd_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      smem)) != cudaSuccess)
-            return e;
-        ring_fwd_tc_kernel<128><<<grid, kThreads, smem, ctx.stream>>>(a);
-    }
-    return cudaGetLastError();
+    if (sh.D == 64)
+        return sh.gathered ? launch<64, true>(a, grid, ctx) : launch<64, false>(a, grid, ctx);
+    return sh.gathered ? launch<128, true>(a, grid, ctx) : launch<128, false>(a, grid, ctx);
 }
 
 }  // namespace rm

@@ -22,6 +22,7 @@ struct AttnShape {
     float scale;
     int window;            // causal left window in keys (query i sees i - window < j <= i); 0 = none
     const void* bounds;    // per-token int4 {lo, hi, imin, imax} of packed documents, or null
+    int gathered;          // forward only: k, v hold all S keys in natural order (all-gather)
 };
 
 // Dynamic work distribution: a persistent kernel's CTAs take work items from a

@@ -21,6 +21,8 @@ _vp, _i, _i64, _f, _sz, _u64 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, c
                                  ctypes.c_size_t, ctypes.c_uint64)
 SIGNATURES = {
     "rm_ring_attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
+    "rm_allgather_attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i,
+                                   _f, _vp]),
     "rm_ring_attn_fwd_window": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                                      _f, _vp]),
     "rm_varlen_bounds_size": (_sz, [_i, _i]),
@@ -106,6 +108,12 @@ def rm_ring_attn_fwd(q, k, v, o, lse, B, H, Hkv, S, D, P, causal, order, dtype, 
                      stream=None):
     return _call("rm_ring_attn_fwd", _p(q), _p(k), _p(v), _p(o), _p(lse), B, H, Hkv, S, D, P,
                  int(causal), order, dtype, scale, _s(stream))
+
+
+def rm_allgather_attn_fwd(q, k_all, v_all, o, lse, B, H, Hkv, S, D, P, causal, order, dtype,
+                          scale, stream=None):
+    return _call("rm_allgather_attn_fwd", _p(q), _p(k_all), _p(v_all), _p(o), _p(lse), B, H, Hkv,
+                 S, D, P, int(causal), order, dtype, scale, _s(stream))
 
 
 def rm_ring_attn_fwd_window(q, k, v, o, lse, B, H, Hkv, S, D, P, window, order, dtype, scale,

@@ -28,7 +28,7 @@ def header_functions():
 def test_header_declares_the_path():
     fns = header_functions()
     for name in ("rm_ring_attn_fwd", "rm_ring_attn_bwd", "rm_ring_attn_bwd_workspace_size",
-                 "rm_ring_attn_fwd_window", "rm_ring_attn_bwd_window",
+                 "rm_ring_attn_fwd_window", "rm_ring_attn_bwd_window", "rm_allgather_attn_fwd",
                  "rm_varlen_bounds", "rm_ring_attn_fwd_varlen", "rm_ring_attn_bwd_varlen",
                  "rm_lse_merge", "rm_ulysses_permute", "rm_ulysses_permute_qkv",
                  "rm_seq_reorder", "rm_check_device_status", "rm_status_string"):
@@ -125,6 +125,26 @@ def test_window_calls_reach_the_device_without_gpu(lib):
                                        None) == 3
     assert lib.rm_ring_attn_fwd_window(A, A, A, A, A, 1, 4, 2, 1024, 64, 4, 5000, 0, 1, 0.125,
                                        None) == 3
+
+
+def test_allgather_validation(lib):
+    def ag(S=1024, D=128, dtype=0, order=1, q=A, Hkv=2):
+        return lib.rm_allgather_attn_fwd(q, A, A, A, A, 1, 4, Hkv, S, D, 4, 1, order, dtype,
+                                         0.088, None)
+    assert ag(dtype=1) == 2                      # the fp32 path has no gathered variant
+    assert ag(dtype=5) == 1
+    assert ag(S=0) == 0                          # empty: nothing to do
+    assert ag(S=1004) == 1                       # shape rules of the ring forward
+    assert ag(D=96) == 2
+    assert ag(q=A + 8) == 1                      # misaligned
+    assert ag(Hkv=3) == 1                        # H % Hkv
+    assert ag(order=9) == 1
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_allgather_call_reaches_the_device_without_gpu(lib):
+    assert lib.rm_allgather_attn_fwd(A, A, A, A, A, 1, 4, 2, 1024, 128, 4, 1, 1, 0, 0.088,
+                                     None) == 3
 
 
 def test_varlen_validation(lib):
