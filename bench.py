@@ -594,7 +594,7 @@ def main():
         line.update({
             "value": value, "unit": "TFLOPS", "ms_per_step": ms_step,
             "pct_of_peak": 100.0 * achieved / peak,
-            "roofline": {"bound": "tensor", "kernel": "ring_fwd_tc_kernel<128>",
+            "roofline": {"bound": "tensor", "kernel": "ring_fwd_tc_kernel<128, false>",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak,
                          "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)",
