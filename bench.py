@@ -44,7 +44,7 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--only", choices=["all", "fwd", "permute", "bwd", "window", "packed",
-                                      "layout", "allgather"],
+                                      "layout", "allgather", "steps"],
                    default="all",
                    help="restrict to one kernel (used for profiling runs)")
     p.add_argument("--skip-cpu", action="store_true", help="skip the CPU oracle baseline")
@@ -467,6 +467,49 @@ def bench_allgather(args, dev, stream):
             "kv_bytes_per_rank": {"ring": 2 * kv_block, "allgather": w.P * kv_block}}
 
 
+def bench_steps(args, dev, stream):
+    """The bench workload as the ranks of a multi-device ring would run it, all
+    on this device: for each of the P ranks, P launches of
+    rm_ring_attn_fwd_step (its queries against one owner block) and P
+    rm_lse_merge folds. The block exchange itself is not part of this (one
+    device); the figure is the cost of splitting the fused ring into steps."""
+    import torch
+    import ring_ulysses_sequence_b200 as rm
+    from ring_ulysses_sequence_b200.synth import WORKLOADS, BENCH_WORKLOAD
+    w = WORKLOADS[BENCH_WORKLOAD]
+    L = w.S // w.P
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed)
+    q, k, v = ((torch.randn(s, generator=g, device=dev) * w.input_scale).to(w.dtype)
+               for s in [(w.P, w.B, w.H, L, w.D), (w.P, w.B, w.Hkv, L, w.D),
+                         (w.P, w.B, w.Hkv, L, w.D)])
+    o_acc = torch.empty((w.P, w.B, w.H, L, w.D), dtype=torch.float32, device=dev)
+    l_acc = torch.empty((w.P, w.B, w.H, L), dtype=torch.float32, device=dev)
+    o_p = torch.empty((w.B, w.H, L, w.D), dtype=torch.float32, device=dev)
+    l_p = torch.empty((w.B, w.H, L), dtype=torch.float32, device=dev)
+
+    def step():
+        with torch.cuda.stream(stream):
+            o_acc.zero_()
+            l_acc.fill_(float("-inf"))
+        for rank in range(w.P):
+            for t in range(w.P):
+                owner = (rank - t) % w.P
+                rm.ring_attn_fwd_step(q[rank], k[owner], v[owner], w.P, rank, owner, w.causal,
+                                      w.order, out=o_p, lse=l_p, stream=stream)
+                rm.lse_merge_(o_acc[rank], l_acc[rank], o_p, l_p, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 20))
+    ms = time_on_stream(step, steps, stream) / steps
+    if rm.native.rm_check_device_status(stream) != 0:
+        raise RuntimeError("device watchdog fired during the step benchmark")
+    return {"workload": w.name, "ms_per_step": ms, "tflops": w.fwd_flops() / ms / 1e9,
+            "launches_per_step": 2 * w.P * w.P + 2, "flops_per_step": w.fwd_flops()}
+
+
 def bench_masked(args, dev, stream, name):
     """Forward with a sparser mask: the 32k GQA layer with a 4096-key causal
     window, or over packed documents."""
@@ -559,6 +602,8 @@ def main():
             out["layout"] = bench_layout(args, dev, stream)
         if rank == 0 and args.only in ("all", "allgather"):
             out["allgather"] = bench_allgather(args, dev, stream)
+        if rank == 0 and args.only in ("all", "steps"):
+            out["steps"] = bench_steps(args, dev, stream)
         if rank == 0 and args.only in ("all", "window"):
             out["window"] = bench_masked(args, dev, stream,
                                          "ring_fwd_bf16_S32k_gqa_causal_zigzag_window4k")
@@ -645,6 +690,17 @@ def main():
                          "frac": x["tflops_attention"] / peaks["bf16_tflops"],
                          "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)",
                          "flops_per_launch": x["flops_per_launch"]}}
+    if "steps" in out:
+        x = out["steps"]
+        extra["ring_attn_fwd_step"] = {
+            "workload": x["workload"], "ms_per_step": x["ms_per_step"], "TFLOPS": x["tflops"],
+            "step": "P ranks x P steps of rm_ring_attn_fwd_step + rm_lse_merge on one device "
+                    "(no block exchange)",
+            "launches_per_step": x["launches_per_step"],
+            "roofline": {"bound": "tensor", "achieved": x["tflops"], "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": x["tflops"] / peaks["bf16_tflops"],
+                         "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)",
+                         "flops_per_step": x["flops_per_step"]}}
     for key, label in (("window", "ring_attn_fwd_window"), ("packed", "ring_attn_fwd_varlen")):
         if key not in out:
             continue

@@ -124,6 +124,40 @@ RM_API rm_status rm_allgather_attn_fwd(const void* q, const void* k_all, const v
                                        float scale, cudaStream_t stream);
 
 /*
+ * rm_ring_attn_fwd_step — one ring step of one rank, for a ring whose ranks
+ * are separate devices.
+ *
+ * "DeDLOC Guide", Step 3 (the local step) and section 3 (the online-softmax
+ * merge of step partials); "Sequence Parallelism III: Ring Attention"
+ * (duoan.github.io): rank `rank` keeps its queries and at each step attends to
+ * the K/V block it holds, which at step t belongs to owner (rank - t) mod P;
+ * the block then moves on to rank + 1. This call computes that step's partial:
+ * softmax attention of the rank's queries over the owner's keys only, with the
+ * causal mask on GLOBAL positions (as rm_ring_attn_fwd). The caller folds the
+ * partials of the P steps with rm_lse_merge, in any order.
+ *
+ *   q_local      [B, H,   L, D]  BF16: rank `rank`'s L = S / P query rows, in
+ *                                its local chunk order (the rank's slice of the
+ *                                rank-major layout)
+ *   k_block,
+ *   v_block      [B, Hkv, L, D]  BF16: owner `owner`'s L rows, local order
+ *   o_part       [B, H,   L, D]  float32, written: the partial, normalised over
+ *                                the visible keys of this block
+ *   lse_part     [B, H,   L]     float32, written: natural log of the partial
+ *                                sum; a row that sees no key of the block gets
+ *                                O = 0, LSE = -inf (the identity of the merge)
+ *   S, P, order  the global layout (S = P * L); 0 <= rank, owner < P.
+ *
+ * Shapes and validation as rm_ring_attn_fwd (S, P and order describe the whole
+ * sequence). FP32 returns RM_ERR_UNSUPPORTED.
+ */
+RM_API rm_status rm_ring_attn_fwd_step(const void* q_local, const void* k_block,
+                                       const void* v_block, float* o_part, float* lse_part, int B,
+                                       int H, int Hkv, int S, int D, int P, int rank, int owner,
+                                       int causal, rm_order order, rm_dtype dtype, float scale,
+                                       cudaStream_t stream);
+
+/*
  * rm_ring_attn_fwd_window — rm_ring_attn_fwd with a causal sliding window.
  *
  * The axolotl-ringmaster README's Status table (phase 4) lists sliding-window

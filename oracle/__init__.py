@@ -243,6 +243,42 @@ def ring_fwd(q, k, v, causal: bool, P: int, order: int, scale: float = None, row
     return o, lse
 
 
+def step_partial(q_local, k_block, v_block, S: int, P: int, order: int, rank: int, owner: int,
+                 causal: bool, scale: float = None):
+    """One ring step's partial ("DeDLOC Guide", Step 3, restricted to one
+    owner's keys): softmax attention of rank `rank`'s queries over the keys of
+    rank `owner`'s block only, causal on GLOBAL positions. A row that sees no
+    key of the block gets (O, LSE) = (0, -inf), the identity of the merge.
+
+    q_local [B,H,L,D], k_block/v_block [B,Hkv,L,D] in the ranks' local order
+    (L = S/P). Plain dense fp64 numpy, written out from the definition; meant
+    for small cases. Returns O [B,H,L,D], LSE [B,H,L] float64.
+    """
+    q, k, v = _f64(q_local), _f64(k_block), _f64(v_block)
+    B, H, L, D = q.shape
+    Hkv = k.shape[1]
+    G = H // Hkv
+    scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
+    pos = rank_major_positions(S, P, order)
+    qpos = pos[rank * L:(rank + 1) * L]
+    kpos = pos[owner * L:(owner + 1) * L]
+    visible = kpos[None, :] <= qpos[:, None] if causal else np.ones((L, L), dtype=bool)
+    o = np.zeros((B, H, L, D))
+    lse = np.full((B, H, L), -np.inf)
+    for b in range(B):
+        for h in range(H):
+            s = np.where(visible, (q[b, h] @ k[b, h // G].T) * scale, -np.inf)
+            seen = visible.any(axis=1)
+            if not seen.any():
+                continue
+            m = s[seen].max(axis=1, keepdims=True)
+            e = np.exp(s[seen] - m)
+            l = e.sum(axis=1, keepdims=True)
+            o[b, h][seen] = (e / l) @ v[b, h // G]
+            lse[b, h][seen] = (m + np.log(l))[:, 0]
+    return o, lse
+
+
 def lse_merge(o_acc, lse_acc, o_part, lse_part):
     """Merge partial (O, LSE) pairs row by row; returns new (O, LSE).
 

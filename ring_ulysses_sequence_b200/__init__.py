@@ -115,6 +115,28 @@ def allgather_attn_fwd(q, k_all, v_all, P, causal=True, order="zigzag", scale=No
     return out, lse
 
 
+def ring_attn_fwd_step(q_local, k_block, v_block, P, rank, owner, causal=True, order="zigzag",
+                       scale=None, out=None, lse=None, stream=None):
+    """One ring step of rank `rank`: its queries q_local [B,H,L,D] against the
+    block k_block/v_block [B,Hkv,L,D] of rank `owner` (L = S / P, local order).
+    Returns the step's partial (O [B,H,L,D] float32, LSE [B,H,L] float32); a row
+    that sees none of the block gets (0, -inf). Fold partials with lse_merge_."""
+    import torch
+    for t, n in ((q_local, "q_local"), (k_block, "k_block"), (v_block, "v_block")):
+        _need(t, n)
+    B, H, L, D = q_local.shape
+    Hkv = k_block.shape[1]
+    if out is None:
+        out = torch.empty(q_local.shape, dtype=torch.float32, device=q_local.device)
+    if lse is None:
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=q_local.device)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    native.rm_ring_attn_fwd_step(q_local, k_block, v_block, out, lse, B, H, Hkv, L * P, D, P,
+                                 rank, owner, causal, _order(order), _dtype_code(q_local), scale,
+                                 stream)
+    return out, lse
+
+
 def ring_attn_bwd(q, k, v, o, lse, dout, P, causal=True, order="zigzag", scale=None,
                   workspace=None, stream=None, window=0, bounds=None):
     """Ring attention backward. Returns fp32 (dQ, dK, dV).

@@ -132,7 +132,7 @@ static rm_status window_arg(int window, int S, int* out) {
 static rm_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse,
                           int B, int H, int Hkv, int S, int D, int P, int causal, int window,
                           const void* bounds, rm_order order, rm_dtype dtype, float scale,
-                          cudaStream_t stream, int gathered = 0) {
+                          cudaStream_t stream, int mode = 0, int rank = 0, int owner = 0) {
     const int tile_q = dtype == RM_DTYPE_BF16 ? 128 : 64;
     rm_status st = check_attn(q, k, v, B, H, Hkv, S, D, P, order, dtype, scale, tile_q);
     if (st != RM_OK) return st;
@@ -141,7 +141,7 @@ static rm_status fwd_impl(const void* q, const void* k, const void* v, void* o, 
     LaunchCtx ctx;
     if ((st = get_ctx(stream, &ctx)) != RM_OK) return st;
     AttnShape sh{B, H, Hkv, S, D, P, causal ? 1 : 0, order == RM_ORDER_ZIGZAG ? 1 : 0, scale,
-                 window, bounds, gathered};
+                 window, bounds, mode, rank, owner};
     cudaError_t e = dtype == RM_DTYPE_BF16
                         ? launch_fwd_tc(sh, q, k, v, o, lse, ctx)
                         : launch_fwd_fp32(sh, static_cast<const float*>(q),
@@ -223,6 +223,16 @@ rm_status rm_allgather_attn_fwd(const void* q, const void* k_all, const void* v_
     if (dtype == RM_DTYPE_FP32) return RM_ERR_UNSUPPORTED;
     return fwd_impl(q, k_all, v_all, o, lse, B, H, Hkv, S, D, P, causal, 0, nullptr, order, dtype,
                     scale, stream, 1);
+}
+
+rm_status rm_ring_attn_fwd_step(const void* q_local, const void* k_block, const void* v_block,
+                                float* o_part, float* lse_part, int B, int H, int Hkv, int S,
+                                int D, int P, int rank, int owner, int causal, rm_order order,
+                                rm_dtype dtype, float scale, cudaStream_t stream) {
+    if (P <= 0 || rank < 0 || rank >= P || owner < 0 || owner >= P) return RM_ERR_INVALID_ARG;
+    if (dtype == RM_DTYPE_FP32) return RM_ERR_UNSUPPORTED;
+    return fwd_impl(q_local, k_block, v_block, o_part, lse_part, B, H, Hkv, S, D, P, causal, 0,
+                    nullptr, order, dtype, scale, stream, 2, rank, owner);
 }
 
 rm_status rm_ring_attn_fwd_window(const void* q, const void* k, const void* v, void* o,

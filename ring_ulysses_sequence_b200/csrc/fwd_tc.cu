@@ -28,11 +28,18 @@
 // runs. O is rescaled only when a row maximum grows by more than 2^8 (in exp2
 // units); the sum l uses the same reference maximum, so the result is exact.
 //
-// The all-gather variant (kGathered; the "allgather" rotater of the
-// axolotl-ringmaster README, Benchmark section: faster, more memory) runs the
-// same kernel with K/V already gathered from every rank into natural token
-// order: each query tile makes one pass over the visible key tiles in
-// position order instead of P ring steps.
+// Three instantiations (kMode):
+//   kRing      all P ranks' queries and all P steps in one launch (K/V of every
+//              rank resident, rank-major).
+//   kGathered  the all-gather variant (the "allgather" rotater of the
+//              axolotl-ringmaster README, Benchmark section: faster, more
+//              memory): K/V gathered from every rank into natural token order;
+//              each query tile makes one pass over its visible key tiles.
+//   kStep      one ring step of one rank, as a rank of a real multi-device ring
+//              runs it: that rank's L local queries against one owner's L-token
+//              K/V block. O (fp32, normalised over this block's keys) and LSE
+//              are the step's partial; a row that sees none of the block gets
+//              (0, -inf), the identity of the (O, LSE) merge.
 #include <algorithm>
 
 #include "common.cuh"
@@ -50,6 +57,7 @@ constexpr int kThreads = 320;
 constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest stale-max factor
+enum Mode : int { kRing = 0, kGathered = 1, kStep = 2 };
 
 template <int D>
 struct Cfg {
@@ -77,6 +85,10 @@ struct TcArgs {
     int n_items;
     float scale, scale_log2;
     RingLayout lay;
+    int q_len;         // rows per head of q, o, lse: S, or L for one step
+    int q_slot0;       // global slot of their first row: 0, or rank * L for one step
+    int kv_len;        // rows per head of k, v: S, or L for one step
+    int owner;         // one step: the rank whose block k, v hold
 };
 
 struct Item {
@@ -86,6 +98,8 @@ struct Item {
 // Work item w -> two query tiles. Items are ordered by the natural position of
 // their queries, latest first when causal (the most key tiles first), with the
 // heads of one position adjacent so that concurrent CTAs share K/V in L2.
+// One step covers only the launching rank's slots, in slot order.
+template <int kMode>
 __device__ __forceinline__ Item decode_item(const TcArgs& a, int w) {
     Item it;
     const int unit_rank = w / a.n_head_units;
@@ -99,7 +113,9 @@ __device__ __forceinline__ Item decode_item(const TcArgs& a, int w) {
     const int U = a.head_pair ? kBM : 2 * kBM;
     const int nu = a.causal ? a.n_units - 1 - unit_rank : unit_rank;
     int slot;
-    if (!a.lay.zigzag || a.lay.c % U == 0)
+    if (kMode == kStep)
+        slot = a.q_slot0 + nu * U;
+    else if (!a.lay.zigzag || a.lay.c % U == 0)
         slot = a.lay.slot_of_pos(nu * U);  // the unit is contiguous in slots too
     else
         slot = nu * U;                     // chunk of one tile: take slot order
@@ -120,8 +136,9 @@ __device__ __forceinline__ Item decode_item(const TcArgs& a, int w) {
 // returned.
 //
 // Gathered variant: the keys are one run of all S positions in natural order
-// (slot = position), visited once.
-template <bool kGathered>
+// (slot = position), visited once. One step: the runs of the owner's block
+// only; kslot is then the row within the block.
+template <int kMode>
 struct KvIter {
     int rank, lo, hi, t, run, u, u_end, s0, p0, kpos;
     __device__ __forceinline__ KvIter(const TcArgs& a, const Item& it)
@@ -132,7 +149,26 @@ struct KvIter {
     // `a` is the kernel's parameter block itself
     __device__ __forceinline__ bool next(const TcArgs& a, int& kslot) {
         const RingLayout& lay = a.lay;
-        if constexpr (kGathered) {
+        if constexpr (kMode == kStep) {
+            while (u >= u_end) {
+                const int runs = lay.zigzag ? 2 : 1;
+                if (run + 1 >= runs) {  // run starts at -1; stays at runs once done
+                    run = runs;
+                    return false;
+                }
+                ++run;
+                const int r = a.owner;
+                const int ctiles = (lay.zigzag ? lay.c : lay.L) / kBN;
+                s0 = run * lay.c;
+                p0 = lay.zigzag ? (run == 0 ? r * lay.c : (2 * lay.P - 1 - r) * lay.c) : r * lay.L;
+                u = max(0, ceil_div128(lo - (kBN - 1) - p0));
+                u_end = min(ctiles, max(((hi - p0) >> 7) + 1, 0));
+            }
+            kpos = p0 + u * kBN;
+            kslot = s0 + u * kBN;
+            ++u;
+            return true;
+        } else if constexpr (kMode == kGathered) {
             if (u >= u_end) {
                 if (run >= 0) return false;  // run starts at -1: one run only
                 run = 0;
@@ -201,7 +237,7 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint3
                 (accumulate || k > 0) ? 1u : 0u);
 }
 
-template <int D, bool kGathered>
+template <int D, int kMode>
 __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_constant__ TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -250,21 +286,24 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
                 int w;
                 ok = item_claim(bars.items, a.work, k, w, wd);
                 if (!ok || w >= a.n_items) break;
-                const Item it = decode_item(a, w);
+                const Item it = decode_item<kMode>(a, w);
+                KvIter<kMode> kv(a, it);
+                int kslot;
+                bool more = kv.next(a, kslot);
+                if (kMode == kStep && !more) continue;  // nothing of this block is visible
                 if (q_iter > 0) ok = mbar_wait(smem_u32(&bars.q_empty), (q_iter - 1) & 1, wd);
                 if (!ok) break;
                 ++q_iter;
                 mbar_arrive_expect_tx(smem_u32(&bars.q_full), 2 * Cfg<D>::kTileBytes);
                 for (int x = 0; x < 2; ++x) {
-                    const int row = ((it.b * a.H) + (x ? it.h1 : it.h0)) * a.S + (x ? it.slot1 : it.slot0);
+                    const int row = ((it.b * a.H) + (x ? it.h1 : it.h0)) * a.q_len +
+                                    (x ? it.slot1 : it.slot0) - a.q_slot0;
                     for (int bx = 0; bx < Cfg<D>::kBoxes; ++bx)
                         tma_load_2d(q_smem + x * Cfg<D>::kTileBytes + bx * Cfg<D>::kBoxBytes, &a.tm_q,
                                     bx * 64, row, smem_u32(&bars.q_full));
                 }
-                KvIter<kGathered> kv(a, it);
-                int kslot;
-                while (ok && kv.next(a, kslot)) {
-                    const int row = (it.b * a.Hkv + it.g) * a.S + kslot;
+                for (; ok && more; more = kv.next(a, kslot)) {
+                    const int row = (it.b * a.Hkv + it.g) * a.kv_len + kslot;
                     for (int which = 0; which < 2 && ok; ++which) {  // K then V
                         const int st = kv_iter % kStages;
                         const uint32_t use = kv_iter / kStages;
@@ -300,10 +339,12 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
                 int w;
                 ok = item_read(bars.items, k, w, false, wd);
                 if (!ok || w >= a.n_items) break;
-                const Item it = decode_item(a, w);
-                KvIter<kGathered> kv(a, it);
+                const Item it = decode_item<kMode>(a, w);
+                KvIter<kMode> kv(a, it);
                 int ks;
-                bool have_cur = kv.next(a, ks);   // tile 0 (every item has one)
+                bool have_cur = kv.next(a, ks);   // tile 0 (every item has one, but
+                if (kMode == kStep && !have_cur)  // in one step it may see none)
+                    continue;
                 bool have_next = kv.next(a, ks);  // tile 1
                 ok = mbar_wait(smem_u32(&bars.q_full), q_iter & 1, wd);
                 if (!ok) break;
@@ -379,9 +420,9 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
             int w;
             ok = item_read(bars.items, k, w, true, wd);
             if (!ok || w >= a.n_items) break;
-            const Item it = decode_item(a, w);
+            const Item it = decode_item<kMode>(a, w);
             float m = -INFINITY, l = 0.f;
-            KvIter<kGathered> kv(a, it);
+            KvIter<kMode> kv(a, it);
             const int qpos = x ? it.pos1 : it.pos0;
             const int2 bf = row_bounds(a.mk, qpos), bl = row_bounds(a.mk, qpos + kBM - 1);
             int kslot, j = 0;
@@ -465,25 +506,52 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
                 ++j;
             }
             if (!ok) break;
-            // epilogue: O / l -> bf16, LSE = m * scale + ln l
+            const int h = x ? it.h1 : it.h0;
+            const int64_t orow = (static_cast<int64_t>(it.b) * a.H + h) * a.q_len +
+                                 (x ? it.slot1 : it.slot0) - a.q_slot0 + r;
+            if constexpr (kMode == kStep) {
+                if (j == 0) {  // the item saw nothing of this block: the merge identity
+                    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.o) + orow * D);
+#pragma unroll 1
+                    for (int c = 0; c < D / 4; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    a.lse[orow] = -INFINITY;
+                    continue;
+                }
+            }
+            // epilogue: O / l -> bf16 (fp32 for one step), LSE = m * scale + ln l
             ok = mbar_wait(smem_u32(&bars.o_full[x]), (o_cnt++) & 1, wd);
             if (!ok) break;
             tc_fence_after();
-            const int h = x ? it.h1 : it.h0;
-            const int64_t orow = (static_cast<int64_t>(it.b) * a.H + h) * a.S + (x ? it.slot1 : it.slot0) + r;
             const float inv = l > 0.f ? 1.0f / l : 0.f;
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + orow * D);
+            if constexpr (kMode == kStep) {
+                float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.o) + orow * D);
 #pragma unroll 1
-            for (int cc = 0; cc < D; cc += 32) {
-                uint32_t ov[32];
-                tmem_ld32(tO + cc, ov);
-                uint32_t pk[16];
+                for (int cc = 0; cc < D; cc += 32) {
+                    uint32_t ov[32];
+                    tmem_ld32(tO + cc, ov);
 #pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    pk[c] = pack_bf16x2(__uint_as_float(ov[2 * c]) * inv, __uint_as_float(ov[2 * c + 1]) * inv);
+                    for (int v4 = 0; v4 < 8; ++v4)
+                        dst[cc / 4 + v4] = make_float4(__uint_as_float(ov[4 * v4]) * inv,
+                                                       __uint_as_float(ov[4 * v4 + 1]) * inv,
+                                                       __uint_as_float(ov[4 * v4 + 2]) * inv,
+                                                       __uint_as_float(ov[4 * v4 + 3]) * inv);
+                }
+            } else {
+                uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + orow * D);
+#pragma unroll 1
+                for (int cc = 0; cc < D; cc += 32) {
+                    uint32_t ov[32];
+                    tmem_ld32(tO + cc, ov);
+                    uint32_t pk[16];
 #pragma unroll
-                for (int v4 = 0; v4 < 4; ++v4)
-                    dst[cc / 8 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+                    for (int c = 0; c < 16; ++c)
+                        pk[c] = pack_bf16x2(__uint_as_float(ov[2 * c]) * inv,
+                                            __uint_as_float(ov[2 * c + 1]) * inv);
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4)
+                        dst[cc / 8 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2],
+                                                      pk[4 * v4 + 3]);
+                }
             }
             a.lse[orow] = l > 0.f ? m * a.scale + logf(l) : -INFINITY;
         }
@@ -496,13 +564,13 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
     }
 }
 
-template <int D, bool kGathered>
+template <int D, int kMode>
 cudaError_t launch(const TcArgs& a, int grid, const LaunchCtx& ctx) {
     constexpr int smem = Cfg<D>::kSmemBytes;
-    cudaError_t e = cudaFuncSetAttribute(ring_fwd_tc_kernel<D, kGathered>,
+    cudaError_t e = cudaFuncSetAttribute(ring_fwd_tc_kernel<D, kMode>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    ring_fwd_tc_kernel<D, kGathered><<<grid, kThreads, smem, ctx.stream>>>(a);
+    ring_fwd_tc_kernel<D, kMode><<<grid, kThreads, smem, ctx.stream>>>(a);
     return cudaGetLastError();
 }
 
@@ -512,8 +580,11 @@ cudaError_t launch_fwd_tc(const AttnShape& sh, const void* q, const void* k, con
                           void* o, float* lse, const LaunchCtx& ctx) {
     TcArgs a{};
     cudaError_t e;
-    const uint64_t qrows = static_cast<uint64_t>(sh.B) * sh.H * sh.S;
-    const uint64_t kvrows = static_cast<uint64_t>(sh.B) * sh.Hkv * sh.S;
+    const bool step = sh.mode == kStep;
+    const int L = sh.S / sh.P;
+    const int len = step ? L : sh.S;  // rows per head of q, k, v (one step: a rank's block)
+    const uint64_t qrows = static_cast<uint64_t>(sh.B) * sh.H * len;
+    const uint64_t kvrows = static_cast<uint64_t>(sh.B) * sh.Hkv * len;
     if ((e = make_tmap_bf16_rows(&a.tm_q, q, qrows, sh.D, kBM, 64)) != cudaSuccess) return e;
     if ((e = make_tmap_bf16_rows(&a.tm_k, k, kvrows, sh.D, kBN, 64)) != cudaSuccess) return e;
     if ((e = make_tmap_bf16_rows(&a.tm_v, v, kvrows, sh.D, kBN, 64)) != cudaSuccess) return e;
@@ -530,17 +601,26 @@ cudaError_t launch_fwd_tc(const AttnShape& sh, const void* q, const void* k, con
     a.G = sh.H / sh.Hkv;
     a.mk = MaskSpec{static_cast<const int4*>(sh.bounds), sh.S, sh.causal, sh.causal ? sh.window : 0};
     a.head_pair = (a.G % 2 == 0) ? 1 : 0;
-    a.n_units = a.head_pair ? sh.S / kBM : sh.S / (2 * kBM);
+    a.n_units = a.head_pair ? len / kBM : len / (2 * kBM);
     a.n_head_units = sh.B * (a.head_pair ? sh.H / 2 : sh.H);
     a.n_items = a.n_units * a.n_head_units;
     a.scale = sh.scale;
     a.scale_log2 = sh.scale * 1.4426950408889634f;
     a.lay = RingLayout{sh.S, sh.P, sh.S / sh.P, sh.zigzag ? sh.S / (2 * sh.P) : sh.S / sh.P,
                        sh.zigzag};
+    a.q_len = len;
+    a.q_slot0 = step ? sh.rank * L : 0;
+    a.kv_len = len;
+    a.owner = step ? sh.owner : 0;
     const int grid = std::min(a.n_items, ctx.num_sms);
-    if (sh.D == 64)
-        return sh.gathered ? launch<64, true>(a, grid, ctx) : launch<64, false>(a, grid, ctx);
-    return sh.gathered ? launch<128, true>(a, grid, ctx) : launch<128, false>(a, grid, ctx);
+    if (sh.D == 64) {
+        if (sh.mode == kStep) return launch<64, kStep>(a, grid, ctx);
+        if (sh.mode == kGathered) return launch<64, kGathered>(a, grid, ctx);
+        return launch<64, kRing>(a, grid, ctx);
+    }
+    if (sh.mode == kStep) return launch<128, kStep>(a, grid, ctx);
+    if (sh.mode == kGathered) return launch<128, kGathered>(a, grid, ctx);
+    return launch<128, kRing>(a, grid, ctx);
 }
 
 }  // namespace rm

@@ -22,7 +22,12 @@ struct AttnShape {
     float scale;
     int window;            // causal left window in keys (query i sees i - window < j <= i); 0 = none
     const void* bounds;    // per-token int4 {lo, hi, imin, imax} of packed documents, or null
-    int gathered;          // forward only: k, v hold all S keys in natural order (all-gather)
+    // Forward only. mode 0: the whole ring (q, k, v rank-major, all S rows);
+    // 1: k, v hold all S keys in natural order (all-gather); 2: one ring step of
+    // rank `rank` (q, o, lse: its L = S / P rows; k, v: the L rows of `owner`'s
+    // block; o is fp32).
+    int mode;
+    int rank, owner;
 };
 
 // Dynamic work distribution: a persistent kernel's CTAs take work items from a
@@ -33,7 +38,7 @@ constexpr int kWorkSlots = 256;
 // Zeroes a fresh counter slot on ctx.stream and returns its address.
 cudaError_t next_work_counter(const LaunchCtx& ctx, int** counter);
 
-// Forward, bf16, tcgen05 tensor cores (fwd_tc.cu).
+// Forward, bf16, tcgen05 tensor cores (fwd_tc.cu). Modes: see AttnShape::mode.
 cudaError_t launch_fwd_tc(const AttnShape& sh, const void* q, const void* k, const void* v,
                           void* o, float* lse, const LaunchCtx& ctx);
 // Forward, fp32 FMA path (fwd_simt.cu).

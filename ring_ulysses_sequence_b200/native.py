@@ -23,6 +23,8 @@ SIGNATURES = {
     "rm_ring_attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "rm_allgather_attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                                    _f, _vp]),
+    "rm_ring_attn_fwd_step": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i,
+                                   _i, _i, _f, _vp]),
     "rm_ring_attn_fwd_window": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                                      _f, _vp]),
     "rm_varlen_bounds_size": (_sz, [_i, _i]),
@@ -114,6 +116,13 @@ def rm_allgather_attn_fwd(q, k_all, v_all, o, lse, B, H, Hkv, S, D, P, causal, o
                           scale, stream=None):
     return _call("rm_allgather_attn_fwd", _p(q), _p(k_all), _p(v_all), _p(o), _p(lse), B, H, Hkv,
                  S, D, P, int(causal), order, dtype, scale, _s(stream))
+
+
+def rm_ring_attn_fwd_step(q_local, k_block, v_block, o_part, lse_part, B, H, Hkv, S, D, P, rank,
+                          owner, causal, order, dtype, scale, stream=None):
+    return _call("rm_ring_attn_fwd_step", _p(q_local), _p(k_block), _p(v_block), _p(o_part),
+                 _p(lse_part), B, H, Hkv, S, D, P, rank, owner, int(causal), order, dtype, scale,
+                 _s(stream))
 
 
 def rm_ring_attn_fwd_window(q, k, v, o, lse, B, H, Hkv, S, D, P, window, order, dtype, scale,

@@ -29,6 +29,7 @@ def test_header_declares_the_path():
     fns = header_functions()
     for name in ("rm_ring_attn_fwd", "rm_ring_attn_bwd", "rm_ring_attn_bwd_workspace_size",
                  "rm_ring_attn_fwd_window", "rm_ring_attn_bwd_window", "rm_allgather_attn_fwd",
+                 "rm_ring_attn_fwd_step",
                  "rm_varlen_bounds", "rm_ring_attn_fwd_varlen", "rm_ring_attn_bwd_varlen",
                  "rm_lse_merge", "rm_ulysses_permute", "rm_ulysses_permute_qkv",
                  "rm_seq_reorder", "rm_check_device_status", "rm_status_string"):
@@ -144,6 +145,24 @@ def test_allgather_validation(lib):
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
 def test_allgather_call_reaches_the_device_without_gpu(lib):
     assert lib.rm_allgather_attn_fwd(A, A, A, A, A, 1, 4, 2, 1024, 128, 4, 1, 1, 0, 0.088,
+                                     None) == 3
+
+
+def test_step_validation(lib):
+    def st(rank=0, owner=1, P=4, dtype=0, S=1024, o=A):
+        return lib.rm_ring_attn_fwd_step(A, A, A, o, A, 1, 4, 2, S, 128, P, rank, owner, 1, 1,
+                                         dtype, 0.088, None)
+    assert st(rank=4) == 1 and st(owner=4) == 1 and st(rank=-1) == 1 and st(owner=-2) == 1
+    assert st(P=0) == 1
+    assert st(dtype=1) == 2                      # the fp32 path has no step variant
+    assert st(S=1004) == 1                       # shape rules of the ring forward
+    assert st(o=A + 4) == 1                      # misaligned output
+    assert st(S=0) == 0                          # empty: nothing to do
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_step_call_reaches_the_device_without_gpu(lib):
+    assert lib.rm_ring_attn_fwd_step(A, A, A, A, A, 1, 4, 2, 1024, 128, 4, 2, 3, 1, 1, 0, 0.088,
                                      None) == 3
 
 

@@ -189,6 +189,50 @@ def test_merge_order_independence_and_empty_partials():
     assert np.all(o == 0) and l[0] == -np.inf
 
 
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("order", [oracle.CONTIGUOUS, oracle.ZIGZAG])
+@pytest.mark.parametrize("P", [1, 2, 3, 4])
+def test_step_partials_fold_to_dense_attention(causal, order, P):
+    # One rank's P step partials (one per owner block), merged in ring order,
+    # are attention over all keys: compared with the textbook numpy attention.
+    S = 24 if P == 3 else 32
+    L, H, Hkv, D = S // P, 4, 2, 8
+    q, k, v = _rand((1, H, S, D), 60 + P), _rand((1, Hkv, S, D), 61), _rand((1, Hkv, S, D), 62)
+    o_ref, l_ref = _np_attention(q, k, v, causal, 1.0 / math.sqrt(D))
+    pos = oracle.rank_major_positions(S, P, order)
+    qr, kr, vr = (x[:, :, pos] for x in (q, k, v))   # rank-major by fancy indexing
+    for rank in range(P):
+        sl = slice(rank * L, (rank + 1) * L)
+        o = np.zeros((H * L, D))
+        l = np.full(H * L, -np.inf)
+        for t in range(P):
+            owner = (rank - t) % P
+            blk = slice(owner * L, (owner + 1) * L)
+            op, lp = oracle.step_partial(qr[:, :, sl], kr[:, :, blk], vr[:, :, blk], S, P, order,
+                                         rank, owner, causal)
+            o, l = oracle.lse_merge(o, l, op.reshape(H * L, D), lp.reshape(H * L))
+        rows = pos[sl]
+        assert np.abs(o.reshape(1, H, L, D) - o_ref[:, :, rows]).max() < 1e-12
+        assert np.abs(l.reshape(1, H, L) - l_ref[:, :, rows]).max() < 1e-12
+
+
+def test_step_partial_special_cases():
+    S, P, D = 32, 4, 4
+    L = S // P
+    q, k, v = _rand((1, 2, L, D), 70), _rand((1, 1, L, D), 71), _rand((1, 1, L, D), 72)
+    # contiguous causal: rank 0's queries precede every key of owner 3 -> all empty
+    o, l = oracle.step_partial(q, k, v, S, P, oracle.CONTIGUOUS, 0, 3, True)
+    assert np.all(o == 0) and np.all(l == -np.inf)
+    # an earlier block is fully visible: plain softmax over its L keys
+    o, l = oracle.step_partial(q, k, v, S, P, oracle.CONTIGUOUS, 3, 1, True)
+    s = (q[0, 0] @ k[0, 0].T) / math.sqrt(D)
+    assert np.abs(l[0, 0] - logsumexp(s, axis=1)).max() < 1e-12
+    # P = 1: the step is the whole attention
+    o1, l1 = oracle.step_partial(q, k, v, L, 1, oracle.ZIGZAG, 0, 0, True)
+    o_ref, l_ref = _np_attention(q, k, v, True, 1.0 / math.sqrt(D))
+    assert np.abs(o1 - o_ref).max() < 1e-12 and np.abs(l1 - l_ref).max() < 1e-12
+
+
 def _loss(q, k, v, dout, causal, scale):
     o, _ = oracle.attn_fwd(q, k, v, causal, scale)
     return float((o * dout).sum())
