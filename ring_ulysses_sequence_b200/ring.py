@@ -44,6 +44,10 @@ def ring_attn_fwd_p2p(q_local, k_local, v_local, causal=True, order="zigzag", sc
     merge(o_acc, lse_acc, o_part, lse_part) (in place) default to the CUDA
     calls; they are parameters so that the exchange can be exercised with
     other arithmetic.
+
+    With NCCL, each process must have made its own device current
+    (torch.cuda.set_device) before the first call, and every rank of the
+    group must call this with blocks of the same shape.
     """
     import torch
     import torch.distributed as dist
