@@ -647,7 +647,10 @@ def main():
                          "frac_of_datasheet_2250": achieved / 2250.0,
                          "flops_per_launch": flops,
                          "traffic": profile_traffic("ring_fwd_tc_S32k_gqa_causal_zigzag.txt",
-                                                    sources)},
+                                                    sources),
+                         "traffic_source": "profiles/ring_fwd_tc_S32k_gqa_causal_zigzag.txt "
+                                           "(null when its source digest is not the current "
+                                           "sources')"},
             "clocks": f["clocks"],
             "gpu_launches": f["launches"],
         })
