@@ -577,50 +577,8 @@ def bench_backward(args, dev, stream):
             "flops_per_step": w.bwd_flops()}
 
 
-def main():
-    args = parse_args()
-    if args.impl == "reference":
-        run_reference(args)
-        return
-    import torch
-    from ring_ulysses_sequence_b200 import multi
-    from ring_ulysses_sequence_b200.synth import BENCH_WORKLOAD, WORKLOADS
-    rank, world, local = multi.env_ranks()
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    multi.init("nccl", timeout_s=120, device=dev)
-    peaks, peak_src = load_peaks()
-    stream = torch.cuda.Stream(device=dev)
-    w = WORKLOADS[BENCH_WORKLOAD]
-    out = {}
-    try:
-        if args.only in ("all", "fwd"):
-            out["fwd"] = bench_forward(w, args, dev, stream)
-        if rank == 0 and args.only in ("all", "permute"):
-            out["permute"] = bench_permute(args, dev, stream)
-        if rank == 0 and args.only in ("all", "layout"):
-            out["layout"] = bench_layout(args, dev, stream)
-        if rank == 0 and args.only in ("all", "allgather"):
-            out["allgather"] = bench_allgather(args, dev, stream)
-        if rank == 0 and args.only in ("all", "steps"):
-            out["steps"] = bench_steps(args, dev, stream)
-        if rank == 0 and args.only in ("all", "window"):
-            out["window"] = bench_masked(args, dev, stream,
-                                         "ring_fwd_bf16_S32k_gqa_causal_zigzag_window4k")
-        if rank == 0 and args.only in ("all", "packed"):
-            out["packed"] = bench_masked(args, dev, stream,
-                                         "ring_fwd_bf16_S32k_gqa_causal_zigzag_packed")
-        if rank == 0 and args.only in ("all", "bwd"):
-            try:
-                out["bwd"] = bench_backward(args, dev, stream)
-            except Exception as e:  # backward not available: say so in the line
-                out["bwd"] = {"unavailable": str(e)[:200]}
-    finally:
-        multi.barrier(dev)
-    if rank != 0:
-        multi.shutdown()
-        return
-
+def build_line(out, w, args, world, peaks, peak_src):
+    """The JSON line (without the CPU baseline) from the measurements in `out`."""
     line = {"metric": METRIC, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic (seeded N(0,1) x 0.5, bf16)",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup}
@@ -729,6 +687,54 @@ def main():
                              "peak_source": f"{peak_src} bf16_tflops_sustained"}}
     if extra:
         line["extra"] = extra
+    return line
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    from ring_ulysses_sequence_b200 import multi
+    from ring_ulysses_sequence_b200.synth import BENCH_WORKLOAD, WORKLOADS
+    rank, world, local = multi.env_ranks()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    multi.init("nccl", timeout_s=120, device=dev)
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.Stream(device=dev)
+    w = WORKLOADS[BENCH_WORKLOAD]
+    out = {}
+    try:
+        if args.only in ("all", "fwd"):
+            out["fwd"] = bench_forward(w, args, dev, stream)
+        if rank == 0 and args.only in ("all", "permute"):
+            out["permute"] = bench_permute(args, dev, stream)
+        if rank == 0 and args.only in ("all", "layout"):
+            out["layout"] = bench_layout(args, dev, stream)
+        if rank == 0 and args.only in ("all", "allgather"):
+            out["allgather"] = bench_allgather(args, dev, stream)
+        if rank == 0 and args.only in ("all", "steps"):
+            out["steps"] = bench_steps(args, dev, stream)
+        if rank == 0 and args.only in ("all", "window"):
+            out["window"] = bench_masked(args, dev, stream,
+                                         "ring_fwd_bf16_S32k_gqa_causal_zigzag_window4k")
+        if rank == 0 and args.only in ("all", "packed"):
+            out["packed"] = bench_masked(args, dev, stream,
+                                         "ring_fwd_bf16_S32k_gqa_causal_zigzag_packed")
+        if rank == 0 and args.only in ("all", "bwd"):
+            try:
+                out["bwd"] = bench_backward(args, dev, stream)
+            except Exception as e:  # backward not available: say so in the line
+                out["bwd"] = {"unavailable": str(e)[:200]}
+    finally:
+        multi.barrier(dev)
+    if rank != 0:
+        multi.shutdown()
+        return
+
+    line = build_line(out, w, args, world, peaks, peak_src)
     if world == 1 and not args.skip_cpu and args.only in ("all", "fwd"):
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line), flush=True)
