@@ -44,7 +44,7 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--only", choices=["all", "fwd", "permute", "bwd", "window", "packed",
-                                      "layout", "allgather", "steps"],
+                                      "layout", "allgather", "steps", "bwdsteps", "exchange"],
                    default="all",
                    help="restrict to one kernel (used for profiling runs)")
     p.add_argument("--skip-cpu", action="store_true", help="skip the CPU oracle baseline")
@@ -251,9 +251,15 @@ def run_reference(args):
 
 
 def workload_config(w):
+    """The workload's config (the same for the GPU arm and the reference arm)."""
+    eb = 2 if "bf16" in w.name else 4
+    bytes_in = (w.B * w.H + 2 * w.B * w.Hkv) * w.S * w.D * eb
+    bytes_out = w.B * w.H * w.S * (w.D * eb + 4)
     return {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.Hkv, "S": w.S, "D": w.D, "P": w.P,
             "order": w.order, "causal": w.causal, "global_batch": w.B, "seq_len": w.S,
-            "parallelism": f"ring P={w.P} simulated per GPU"}
+            "parallelism": f"ring P={w.P} simulated per GPU",
+            "l2": f"inputs {bytes_in / 1e6:.0f} MB + outputs {bytes_out / 1e6:.0f} MB "
+                  f"> {L2_BYTES >> 20} MiB L2 (no flush)"}
 
 
 # ---------------------------------------------------------------------------
@@ -488,10 +494,22 @@ def bench_steps(args, dev, stream):
     o_p = torch.empty((w.B, w.H, L, w.D), dtype=torch.float32, device=dev)
     l_p = torch.empty((w.B, w.H, L), dtype=torch.float32, device=dev)
 
-    def step():
+    def reset():
         with torch.cuda.stream(stream):
             o_acc.zero_()
             l_acc.fill_(float("-inf"))
+
+    def step():  # the fused call: each step folds straight into the running pair
+        reset()
+        for rank in range(w.P):
+            for t in range(w.P):
+                owner = (rank - t) % w.P
+                rm.ring_attn_fwd_step_merge(q[rank], k[owner], v[owner], o_acc[rank],
+                                            l_acc[rank], w.P, rank, owner, w.causal, w.order,
+                                            stream=stream)
+
+    def step_two_calls():  # the partial written out, then merged by rm_lse_merge
+        reset()
         for rank in range(w.P):
             for t in range(w.P):
                 owner = (rank - t) % w.P
@@ -499,15 +517,107 @@ def bench_steps(args, dev, stream):
                                       w.order, out=o_p, lse=l_p, stream=stream)
                 rm.lse_merge_(o_acc[rank], l_acc[rank], o_p, l_p, stream=stream)
 
-    for _ in range(max(3, args.warmup)):
-        step()
+    for fn in (step, step_two_calls):
+        for _ in range(max(3, args.warmup)):
+            fn()
     torch.cuda.synchronize()
     steps = max(3, min(args.steps, 20))
     ms = time_on_stream(step, steps, stream) / steps
+    ms2 = time_on_stream(step_two_calls, steps, stream) / steps
     if rm.native.rm_check_device_status(stream) != 0:
         raise RuntimeError("device watchdog fired during the step benchmark")
     return {"workload": w.name, "ms_per_step": ms, "tflops": w.fwd_flops() / ms / 1e9,
-            "launches_per_step": 2 * w.P * w.P + 2, "flops_per_step": w.fwd_flops()}
+            "launches_per_step": w.P * w.P + 2, "flops_per_step": w.fwd_flops(),
+            "ms_per_step_two_calls": ms2, "tflops_two_calls": w.fwd_flops() / ms2 / 1e9}
+
+
+def bench_bwd_steps(args, dev, stream):
+    """The backward of the bench workload as the ranks of a multi-device ring
+    would run it, all on this device: per rank one rm_ring_attn_bwd_delta, and
+    P rm_ring_attn_bwd_step launches in the reverse ring's schedule (dQ
+    accumulating on the rank, dK/dV on the block). No exchange (one device)."""
+    import torch
+    import ring_ulysses_sequence_b200 as rm
+    from ring_ulysses_sequence_b200.synth import WORKLOADS, BENCH_WORKLOAD
+    w = WORKLOADS[BENCH_WORKLOAD]
+    L = w.S // w.P
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed)
+    q, k, v, do = ((torch.randn(s, generator=g, device=dev) * w.input_scale).to(w.dtype)
+                   for s in [(w.P, w.B, w.H, L, w.D), (w.P, w.B, w.Hkv, L, w.D),
+                             (w.P, w.B, w.Hkv, L, w.D), (w.P, w.B, w.H, L, w.D)])
+    qr, kr, vr = (x.permute(1, 2, 0, 3, 4).reshape(w.B, x.shape[2], w.S, w.D).contiguous()
+                  for x in (q, k, v))
+    o, lse = rm.ring_attn_fwd(qr, kr, vr, w.P, w.causal, w.order, stream=stream)
+    o = o.reshape(w.B, w.H, w.P, L, w.D).permute(2, 0, 1, 3, 4).contiguous()
+    lse = lse.reshape(w.B, w.H, w.P, L).permute(2, 0, 1, 3).contiguous()
+    delta = torch.empty_like(lse)
+    dq = torch.empty((w.P, w.B, w.H, L, w.D), dtype=torch.float32, device=dev)
+    dk = torch.empty((w.P, w.B, w.Hkv, L, w.D), dtype=torch.float32, device=dev)
+    dv = torch.empty_like(dk)
+
+    def step():
+        with torch.cuda.stream(stream):
+            dq.zero_()
+            dk.zero_()
+            dv.zero_()
+        for rank in range(w.P):
+            rm.ring_attn_bwd_delta(o[rank], do[rank], out=delta[rank], stream=stream)
+        for t in range(w.P):
+            for rank in range(w.P):
+                owner = (rank - t) % w.P
+                rm.ring_attn_bwd_step(q[rank], k[owner], v[owner], lse[rank], delta[rank],
+                                      do[rank], dq[rank], dk[owner], dv[owner], w.P, rank, owner,
+                                      w.causal, w.order, stream=stream)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    steps = max(2, min(args.steps, 10))
+    ms = time_on_stream(step, steps, stream) / steps
+    if rm.native.rm_check_device_status(stream) != 0:
+        raise RuntimeError("device watchdog fired during the backward step benchmark")
+    return {"workload": w.name, "ms_per_step": ms, "tflops": w.bwd_flops() / ms / 1e9,
+            "launches_per_step": w.P * w.P + w.P + 3, "flops_per_step": w.bwd_flops()}
+
+
+def bench_exchange(args, dev, stream):
+    """The Ulysses exchange-buffer kernels on the 131072-token USP workload's
+    shards (U = 4 x R = 4: 16 devices of 8192 tokens): every device's Q, K, V
+    packed into its send buffer, and every receive buffer unpacked into the
+    device's head shards, 32 launches on this device (the all-to-all between
+    them is NCCL's and not part of this)."""
+    import torch
+    import ring_ulysses_sequence_b200 as rm
+    from ring_ulysses_sequence_b200.synth import WORKLOADS
+    w = WORKLOADS["usp_fwd_bf16_S128k_u4r4"]
+    U, R = w.ulysses, w.P
+    n = U * R
+    s = w.S // n
+    shards = [[torch.randn((w.B, s, h, w.D), device=dev).to(w.dtype) for h in (w.H, w.Hkv, w.Hkv)]
+              for _ in range(n)]
+    heads = [w.H, w.Hkv, w.Hkv]
+    bufs = [torch.empty((w.H + 2 * w.Hkv) * w.B * s * w.D, device=dev, dtype=w.dtype)
+            for _ in range(n)]
+    outs = [[torch.empty((w.B, h // U, U * s, w.D), device=dev, dtype=w.dtype) for h in heads]
+            for _ in range(n)]
+
+    def step():
+        for i in range(n):
+            rm.ulysses_pack(shards[i], U, "seq_to_head", buf=bufs[i], stream=stream)
+        for i in range(n):
+            rm.ulysses_unpack(bufs[i], U, heads, w.B, s, w.D, "seq_to_head", outs=outs[i],
+                              stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            step()
+    torch.cuda.synchronize()
+    steps = max(5, min(args.steps, 50))
+    ms = time_on_stream(step, steps, stream) / steps
+    moved = 2 * 2 * sum(b.numel() * b.element_size() for b in bufs)  # pack + unpack, read + write
+    return {"workload": w.name, "ms_per_step": ms, "bytes_per_step": moved,
+            "gbs": moved / ms / 1e6, "launches_per_step": 2 * n}
 
 
 def bench_masked(args, dev, stream, name):
@@ -573,6 +683,8 @@ def bench_backward(args, dev, stream):
     torch.cuda.synchronize()
     steps = max(2, min(args.steps, 10))
     ms = time_on_stream(step, steps, stream) / steps
+    if rm.native.rm_check_device_status(stream) != 0:
+        raise RuntimeError("device watchdog fired during the backward benchmark")
     return {"workload": w.name, "ms_per_step": ms, "tflops": w.bwd_flops() / ms / 1e9,
             "flops_per_step": w.bwd_flops()}
 
@@ -588,15 +700,19 @@ def build_line(out, w, args, world, peaks, peak_src):
         ms_step = f["ms_total"] / args.steps
         flops = w.fwd_flops()
         value = world * flops * args.steps / (f["ms_total"] * 1e-3) / 1e12
-        cfg["l2"] = (f"inputs {f['bytes_in'] / 1e6:.0f} MB + outputs {f['bytes_out'] / 1e6:.0f} MB "
-                     f"> {L2_BYTES >> 20} MiB L2 (no flush)")
         sources = ["ring_ulysses_sequence_b200/csrc/fwd_tc.cu",
                    "ring_ulysses_sequence_b200/csrc/common.cuh"]
         peak = peaks["bf16_tflops"]
         achieved = flops / (ms_step * 1e-3) / 1e12
         line.update({
             "value": value, "unit": "TFLOPS", "ms_per_step": ms_step,
+            # the denominator is the MEASURED dense bf16 GEMM rate of this pool's
+            # B200s (an achieved-GEMM ceiling), not NVIDIA's datasheet figure;
+            # both fractions are given
             "pct_of_peak": 100.0 * achieved / peak,
+            "pct_of_peak_basis": f"{peak_src} bf16 GEMM ceiling {peak} TFLOPS "
+                                 "(torch.matmul 8192^3 burst on this pool's B200s)",
+            "pct_of_datasheet_dense_peak": 100.0 * achieved / 2250.0,
             "roofline": {"bound": "tensor", "kernel": "ring_fwd_tc_kernel<128, false>",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak,
@@ -655,13 +771,38 @@ def build_line(out, w, args, world, peaks, peak_src):
         x = out["steps"]
         extra["ring_attn_fwd_step"] = {
             "workload": x["workload"], "ms_per_step": x["ms_per_step"], "TFLOPS": x["tflops"],
-            "step": "P ranks x P steps of rm_ring_attn_fwd_step + rm_lse_merge on one device "
+            "step": "P ranks x P steps of rm_ring_attn_fwd_step_merge on one device "
                     "(no block exchange)",
             "launches_per_step": x["launches_per_step"],
+            "ms_per_step_two_calls": x["ms_per_step_two_calls"],
+            "TFLOPS_two_calls": x["tflops_two_calls"],
             "roofline": {"bound": "tensor", "achieved": x["tflops"], "peak": peaks["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": x["tflops"] / peaks["bf16_tflops"],
                          "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)",
                          "flops_per_step": x["flops_per_step"]}}
+    if "bwdsteps" in out:
+        x = out["bwdsteps"]
+        extra["ring_attn_bwd_step"] = {
+            "workload": x["workload"], "ms_per_step": x["ms_per_step"], "TFLOPS": x["tflops"],
+            "step": "per rank rm_ring_attn_bwd_delta, then P x P rm_ring_attn_bwd_step in the "
+                    "reverse ring's schedule on one device (no exchange)",
+            "launches_per_step": x["launches_per_step"],
+            "roofline": {"bound": "tensor", "achieved": x["tflops"],
+                         "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                         "frac": x["tflops"] / peaks["bf16_tflops_sustained"],
+                         "peak_source": f"{peak_src} bf16_tflops_sustained",
+                         "flops_per_step": x["flops_per_step"]}}
+    if "exchange" in out:
+        x = out["exchange"]
+        extra["ulysses_pack_unpack"] = {
+            "workload": x["workload"], "ms_per_step": x["ms_per_step"], "GB/s": x["gbs"],
+            "step": "16 devices' Q/K/V packed into send buffers + 16 receive buffers unpacked "
+                    "(rm_ulysses_pack / rm_ulysses_unpack, SEQ_TO_HEAD)",
+            "launches_per_step": x["launches_per_step"],
+            "roofline": {"bound": "hbm", "achieved": x["gbs"], "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": x["gbs"] / peaks["hbm_gbs"],
+                         "peak_source": f"{peak_src} hbm_gbs",
+                         "bytes_per_step": x["bytes_per_step"]}}
     for key, label in (("window", "ring_attn_fwd_window"), ("packed", "ring_attn_fwd_varlen")):
         if key not in out:
             continue
@@ -717,6 +858,10 @@ def main():
             out["allgather"] = bench_allgather(args, dev, stream)
         if rank == 0 and args.only in ("all", "steps"):
             out["steps"] = bench_steps(args, dev, stream)
+        if rank == 0 and args.only in ("all", "bwdsteps"):
+            out["bwdsteps"] = bench_bwd_steps(args, dev, stream)
+        if rank == 0 and args.only in ("all", "exchange"):
+            out["exchange"] = bench_exchange(args, dev, stream)
         if rank == 0 and args.only in ("all", "window"):
             out["window"] = bench_masked(args, dev, stream,
                                          "ring_fwd_bf16_S32k_gqa_causal_zigzag_window4k")

@@ -158,6 +158,32 @@ RM_API rm_status rm_ring_attn_fwd_step(const void* q_local, const void* k_block,
                                        cudaStream_t stream);
 
 /*
+ * rm_ring_attn_fwd_step_merge — rm_ring_attn_fwd_step folded straight into the
+ * rank's running (O, LSE) pair, so that no partial is written.
+ *
+ * "DeDLOC Guide", section 3 (the alpha/beta rescaling of step partials) and
+ * Step 3: with a = lse_acc and b the step's LSE, M = max(a, b),
+ *   O_acc <- (e^(a-M) O_acc + e^(b-M) O_step) / (e^(a-M) + e^(b-M)),
+ *   lse_acc <- M + ln(e^(a-M) + e^(b-M)).
+ * The same result as rm_ring_attn_fwd_step followed by rm_lse_merge (up to
+ * fp32 rounding order), in one launch and without the partial's round trip
+ * through memory.
+ *
+ *   q_local, k_block, v_block, B..order, dtype, scale : as rm_ring_attn_fwd_step
+ *   o_acc   [B, H, L, D] float32, read and written: the running output
+ *   lse_acc [B, H, L]    float32, read and written: the running LSE
+ * Start a ring with o_acc = 0 and lse_acc = -inf (the empty pair) and call this
+ * once per step, in any order of owners. Rows that see no key of the block keep
+ * their pair unchanged. After the P steps of a rank, (o_acc, lse_acc) is its
+ * attention output and LSE. Shapes and validation as rm_ring_attn_fwd_step.
+ */
+RM_API rm_status rm_ring_attn_fwd_step_merge(const void* q_local, const void* k_block,
+                                             const void* v_block, float* o_acc, float* lse_acc,
+                                             int B, int H, int Hkv, int S, int D, int P, int rank,
+                                             int owner, int causal, rm_order order,
+                                             rm_dtype dtype, float scale, cudaStream_t stream);
+
+/*
  * rm_ring_attn_fwd_window — rm_ring_attn_fwd with a causal sliding window.
  *
  * The axolotl-ringmaster README's Status table (phase 4) lists sliding-window
@@ -311,6 +337,60 @@ RM_API rm_status rm_ring_attn_bwd_noalloc(const void* q, const void* k, const vo
                                           rm_dtype dtype, float scale, cudaStream_t stream);
 
 /*
+ * rm_ring_attn_bwd_delta — Delta_i = <dO_i, O_i> (fp32) for rows of D values:
+ * the per-row term of the backward's dS_ij = P_ij (<dO_i, v_j> - Delta_i)
+ * (the gradient stated at rm_ring_attn_bwd). A rank of a ring across devices
+ * computes it once for its own rows and passes it to every
+ * rm_ring_attn_bwd_step of the backward.
+ *
+ *   o     [rows, D] o_dtype (BF16, or FP32 as rm_ring_attn_fwd_step_merge
+ *                   accumulates it)
+ *   dout  [rows, D] BF16
+ *   delta [rows]    float32, written
+ * D in {64, 128} (else RM_ERR_UNSUPPORTED); rows >= 0.
+ */
+RM_API rm_status rm_ring_attn_bwd_delta(const void* o, const void* dout, float* delta,
+                                        int64_t rows, int D, rm_dtype o_dtype,
+                                        cudaStream_t stream);
+
+/*
+ * rm_ring_attn_bwd_step — one step of the backward of a ring whose ranks are
+ * separate devices (axolotl-ringmaster README, Benchmark section: the p2p
+ * rotater's flash-style reverse-ring backward, gradients accumulated in fp32
+ * across ring steps).
+ *
+ * The gradients of rm_ring_attn_bwd restricted to the pairs (query of rank
+ * `rank`, key of owner `owner`'s block): rank `rank` holds its queries and the
+ * block of `owner`, and this call ADDS
+ *   dq_local += scale sum_{j in block} dS_ij k_j      (the rank's rows)
+ *   dk_block += scale sum_{i of rank} dS_ij q_i       (the block's rows)
+ *   dv_block +=       sum_{i of rank} P_ij dO_i
+ * with P_ij = exp(scale q_i.k_j - LSE_i) over the pairs the causal mask (global
+ * positions) leaves visible. Over the P steps a rank's dq_local collects every
+ * owner's part, and a block's dk/dv, travelling with it, every rank's part.
+ *
+ *   q_local, dout_local [B, H, L, D]  BF16, the rank's rows (local order)
+ *   lse_local           [B, H, L]     float32, the rank's final forward LSE
+ *   delta_local         [B, H, L]     float32, rm_ring_attn_bwd_delta of the
+ *                                     rank's O and dO
+ *   k_block, v_block    [B, Hkv, L, D] BF16, owner `owner`'s rows
+ *   dq_local            [B, H, L, D]  float32, read and written
+ *   dk_block, dv_block  [B, Hkv, L, D] float32, read and written
+ *   S, P, rank, owner, causal, order, scale : as rm_ring_attn_fwd_step
+ * Zero the three gradient arrays before the first step. Tiles that see nothing
+ * of the other side are not touched; every element is updated by one thread
+ * per call, so the sums are deterministic. Shapes and validation as
+ * rm_ring_attn_bwd (BF16, D in {64, 128}).
+ */
+RM_API rm_status rm_ring_attn_bwd_step(const void* q_local, const void* k_block,
+                                       const void* v_block, const float* lse_local,
+                                       const float* delta_local, const void* dout_local,
+                                       float* dq_local, float* dk_block, float* dv_block, int B,
+                                       int H, int Hkv, int S, int D, int P, int rank, int owner,
+                                       int causal, rm_order order, rm_dtype dtype, float scale,
+                                       cudaStream_t stream);
+
+/*
  * rm_lse_merge — fold one partial (O, LSE) into a running pair, row by row,
  * in place ("DeDLOC Guide", section 3 alpha/beta rescaling, in the
  * normalised-output form of Step 3's merge):
@@ -349,6 +429,54 @@ RM_API rm_status rm_ulysses_permute_qkv(const void* q_src, const void* k_src, co
                                  void* q_dst, void* k_dst, void* v_dst, int B, int S, int H,
                                  int Hkv, int D, int U, int R, int elem_bytes,
                                  rm_permute_dir dir, cudaStream_t stream);
+
+/*
+ * rm_ulysses_buffer_size / rm_ulysses_pack / rm_ulysses_unpack — one device's
+ * side of the DeepSpeed-Ulysses all-to-all when the U devices of a Ulysses
+ * group are separate GPUs ("Sequence Parallelism II: DeepSpeed Ulysses and
+ * All-to-All Attention": before the exchange a device has all heads of its
+ * tokens, after it all tokens of its heads; axolotl-ringmaster README: the
+ * Ulysses leg exchanges K and V together, and Ulysses is capped by the
+ * KV-head count).
+ *
+ * Device u of the group holds s = S_group / U consecutive tokens (its
+ * sequence shard). The exchange buffer is U equal chunks, chunk u' for
+ * (pack) or from (unpack) device u'; a collective all-to-all with equal
+ * splits (ncclSend/ncclRecv pairs, torch.distributed.all_to_all_single) moves
+ * chunk u' of every device to device u'. Inside a chunk the tensors follow
+ * one another, tensor x as [B, s, heads[x] / U, D]: the sender's s tokens of
+ * the receiver's heads. Up to three tensors (Q, K, V; or O alone) share one
+ * buffer, so one collective moves them all.
+ *   sequence shard of tensor x: [B, s, heads[x], D]        (device's tokens)
+ *   head shard of tensor x:     [B, heads[x]/U, U*s, D]    (device's heads,
+ *       token u'*s + t = token t of device u', i.e. the group's tokens in order)
+ * Device u's head shard holds heads [u*heads/U, (u+1)*heads/U).
+ *
+ *   rm_ulysses_pack   SEQ_TO_HEAD: tensors = sequence shards -> send_buf
+ *                     HEAD_TO_SEQ: tensors = head shards     -> send_buf
+ *   rm_ulysses_unpack SEQ_TO_HEAD: recv_buf -> tensors = head shards
+ *                     HEAD_TO_SEQ: recv_buf -> tensors = sequence shards
+ * So pack(SEQ_TO_HEAD), all-to-all, unpack(SEQ_TO_HEAD) turns every device's
+ * sequence shard into its head shard, and the HEAD_TO_SEQ pair undoes it.
+ *
+ *   tensors, heads : HOST arrays of ntensors (1..3) device pointers and head
+ *                    counts; heads[x] % U == 0
+ *   send_buf / recv_buf : device buffer of rm_ulysses_buffer_size(heads,
+ *                    ntensors, B, s, D, elem_bytes) bytes, not overlapping any
+ *                    tensor, 16-byte aligned like every pointer here
+ *   elem_bytes in {1, 2, 4, 8}. Bit-exact data movement (HBM-bound).
+ * rm_ulysses_buffer_size returns 0 for invalid arguments.
+ */
+RM_API size_t rm_ulysses_buffer_size(const int* heads, int ntensors, int B, int s, int D,
+                                     int elem_bytes);
+
+RM_API rm_status rm_ulysses_pack(const void* const* tensors, const int* heads, int ntensors,
+                                 void* send_buf, int B, int s, int D, int U, int elem_bytes,
+                                 rm_permute_dir dir, cudaStream_t stream);
+
+RM_API rm_status rm_ulysses_unpack(const void* recv_buf, void* const* tensors, const int* heads,
+                                   int ntensors, int B, int s, int D, int U, int elem_bytes,
+                                   rm_permute_dir dir, cudaStream_t stream);
 
 /*
  * rm_seq_reorder — natural token order <-> rank-major ring order along S.

@@ -279,6 +279,49 @@ def step_partial(q_local, k_block, v_block, S: int, P: int, order: int, rank: in
     return o, lse
 
 
+def step_bwd_partial(q_local, k_block, v_block, dout_local, lse_local, delta_local, S: int,
+                     P: int, order: int, rank: int, owner: int, causal: bool,
+                     scale: float = None):
+    """One ring step's share of the gradients (the backward of L = sum(dO * O)
+    restricted to the pairs (query of rank `rank`, key of owner `owner`'s
+    block); axolotl-ringmaster README, Benchmark: the reverse-ring backward).
+    With P_ij = exp(scale q_i.k_j - LSE_i) over the visible pairs and
+    Delta_i = <dO_i, O_i> of the FULL attention (both inputs here):
+      dV_j = sum_i P_ij dO_i,  dS_ij = P_ij (<dO_i, v_j> - Delta_i),
+      dQ_i = scale sum_j dS_ij k_j,  dK_j = scale sum_i dS_ij q_i,
+    KV gradients summed over the G heads that share a KV head.
+
+    q_local, dout_local [B,H,L,D], k_block, v_block [B,Hkv,L,D] in local
+    order; lse_local, delta_local [B,H,L]. Plain dense fp64 numpy, written
+    out from the definition; meant for small cases. Returns (dQ [B,H,L,D],
+    dK [B,Hkv,L,D], dV [B,Hkv,L,D]) float64.
+    """
+    q, k, v, do = _f64(q_local), _f64(k_block), _f64(v_block), _f64(dout_local)
+    lse, delta = _f64(lse_local), _f64(delta_local)
+    B, H, L, D = q.shape
+    Hkv = k.shape[1]
+    G = H // Hkv
+    scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
+    pos = rank_major_positions(S, P, order)
+    qpos = pos[rank * L:(rank + 1) * L]
+    kpos = pos[owner * L:(owner + 1) * L]
+    visible = kpos[None, :] <= qpos[:, None] if causal else np.ones((L, L), dtype=bool)
+    dq = np.zeros((B, H, L, D))
+    dk = np.zeros((B, Hkv, L, D))
+    dv = np.zeros((B, Hkv, L, D))
+    for b in range(B):
+        for h in range(H):
+            g = h // G
+            s = (q[b, h] @ k[b, g].T) * scale
+            p = np.where(visible, np.exp(s - lse[b, h][:, None]), 0.0)
+            dp = do[b, h] @ v[b, g].T
+            ds = p * (dp - delta[b, h][:, None])
+            dq[b, h] = scale * (ds @ k[b, g])
+            dk[b, g] += scale * (ds.T @ q[b, h])
+            dv[b, g] += p.T @ do[b, h]
+    return dq, dk, dv
+
+
 def lse_merge(o_acc, lse_acc, o_part, lse_part):
     """Merge partial (O, LSE) pairs row by row; returns new (O, LSE).
 

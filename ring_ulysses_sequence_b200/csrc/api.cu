@@ -132,7 +132,8 @@ static rm_status window_arg(int window, int S, int* out) {
 static rm_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse,
                           int B, int H, int Hkv, int S, int D, int P, int causal, int window,
                           const void* bounds, rm_order order, rm_dtype dtype, float scale,
-                          cudaStream_t stream, int mode = 0, int rank = 0, int owner = 0) {
+                          cudaStream_t stream, int mode = 0, int rank = 0, int owner = 0,
+                          int merge = 0) {
     const int tile_q = dtype == RM_DTYPE_BF16 ? 128 : 64;
     rm_status st = check_attn(q, k, v, B, H, Hkv, S, D, P, order, dtype, scale, tile_q);
     if (st != RM_OK) return st;
@@ -141,7 +142,7 @@ static rm_status fwd_impl(const void* q, const void* k, const void* v, void* o, 
     LaunchCtx ctx;
     if ((st = get_ctx(stream, &ctx)) != RM_OK) return st;
     AttnShape sh{B, H, Hkv, S, D, P, causal ? 1 : 0, order == RM_ORDER_ZIGZAG ? 1 : 0, scale,
-                 window, bounds, mode, rank, owner};
+                 window, bounds, mode, rank, owner, merge};
     cudaError_t e = dtype == RM_DTYPE_BF16
                         ? launch_fwd_tc(sh, q, k, v, o, lse, ctx)
                         : launch_fwd_fp32(sh, static_cast<const float*>(q),
@@ -233,6 +234,17 @@ rm_status rm_ring_attn_fwd_step(const void* q_local, const void* k_block, const 
     if (dtype == RM_DTYPE_FP32) return RM_ERR_UNSUPPORTED;
     return fwd_impl(q_local, k_block, v_block, o_part, lse_part, B, H, Hkv, S, D, P, causal, 0,
                     nullptr, order, dtype, scale, stream, 2, rank, owner);
+}
+
+rm_status rm_ring_attn_fwd_step_merge(const void* q_local, const void* k_block,
+                                      const void* v_block, float* o_acc, float* lse_acc, int B,
+                                      int H, int Hkv, int S, int D, int P, int rank, int owner,
+                                      int causal, rm_order order, rm_dtype dtype, float scale,
+                                      cudaStream_t stream) {
+    if (P <= 0 || rank < 0 || rank >= P || owner < 0 || owner >= P) return RM_ERR_INVALID_ARG;
+    if (dtype == RM_DTYPE_FP32) return RM_ERR_UNSUPPORTED;
+    return fwd_impl(q_local, k_block, v_block, o_acc, lse_acc, B, H, Hkv, S, D, P, causal, 0,
+                    nullptr, order, dtype, scale, stream, 2, rank, owner, 1);
 }
 
 rm_status rm_ring_attn_fwd_window(const void* q, const void* k, const void* v, void* o,
@@ -376,6 +388,45 @@ rm_status rm_ring_attn_bwd_noalloc(const void* q, const void* k, const void* v, 
     return e == cudaSuccess ? RM_OK : cuda_fail(e);
 }
 
+rm_status rm_ring_attn_bwd_delta(const void* o, const void* dout, float* delta, int64_t rows,
+                                 int D, rm_dtype o_dtype, cudaStream_t stream) {
+    if (rows < 0 || D <= 0) return RM_ERR_INVALID_ARG;
+    if (o_dtype != RM_DTYPE_BF16 && o_dtype != RM_DTYPE_FP32) return RM_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return RM_ERR_UNSUPPORTED;
+    if (rows == 0) return RM_OK;
+    if (!o || !dout || !delta || !aligned16(o) || !aligned16(dout) || !aligned16(delta))
+        return RM_ERR_INVALID_ARG;
+    LaunchCtx ctx;
+    rm_status st = get_ctx(stream, &ctx);
+    if (st != RM_OK) return st;
+    cudaError_t e = launch_bwd_delta(o, o_dtype == RM_DTYPE_FP32, dout, delta, rows, D, ctx);
+    return e == cudaSuccess ? RM_OK : cuda_fail(e);
+}
+
+rm_status rm_ring_attn_bwd_step(const void* q_local, const void* k_block, const void* v_block,
+                                const float* lse_local, const float* delta_local,
+                                const void* dout_local, float* dq_local, float* dk_block,
+                                float* dv_block, int B, int H, int Hkv, int S, int D, int P,
+                                int rank, int owner, int causal, rm_order order, rm_dtype dtype,
+                                float scale, cudaStream_t stream) {
+    if (P <= 0 || rank < 0 || rank >= P || owner < 0 || owner >= P) return RM_ERR_INVALID_ARG;
+    rm_status st = check_attn(q_local, k_block, v_block, B, H, Hkv, S, D, P, order, dtype, scale,
+                              128);
+    if (st != RM_OK) return st;
+    if (dtype != RM_DTYPE_BF16) return RM_ERR_UNSUPPORTED;
+    if (B == 0 || S == 0) return RM_OK;
+    const void* ptrs[] = {lse_local, delta_local, dout_local, dq_local, dk_block, dv_block};
+    for (const void* p : ptrs)
+        if (!p || !aligned16(p)) return RM_ERR_INVALID_ARG;
+    LaunchCtx ctx;
+    if ((st = get_ctx(stream, &ctx)) != RM_OK) return st;
+    AttnShape sh{B, H, Hkv, S, D, P, causal ? 1 : 0, order == RM_ORDER_ZIGZAG ? 1 : 0, scale, 0,
+                 nullptr, 2, rank, owner, 0};
+    cudaError_t e = launch_bwd(sh, q_local, k_block, v_block, nullptr, lse_local, dout_local,
+                               dq_local, dk_block, dv_block, const_cast<float*>(delta_local), ctx);
+    return e == cudaSuccess ? RM_OK : cuda_fail(e);
+}
+
 rm_status rm_lse_merge(float* o_acc, float* lse_acc, const float* o_part, const float* lse_part,
                        int64_t rows, int D, cudaStream_t stream) {
     if (rows < 0 || D <= 0) return RM_ERR_INVALID_ARG;
@@ -430,6 +481,56 @@ rm_status rm_ulysses_permute_qkv(const void* q_src, const void* k_src, const voi
     PermuteTensor t[3] = {{q_src, q_dst, H}, {k_src, k_dst, Hkv}, {v_src, v_dst, Hkv}};
     cudaError_t e = launch_ulysses_permute(t, 3, B, S, D, elem_bytes, dir == RM_HEAD_TO_SEQ, ctx);
     return e == cudaSuccess ? RM_OK : cuda_fail(e);
+}
+
+static rm_status ulysses_exchange(const void* const* tensors, const int* heads, int ntensors,
+                                  void* buf, int B, int s, int D, int U, int elem_bytes,
+                                  rm_permute_dir dir, int pack, cudaStream_t stream) {
+    if (B < 0 || s < 0 || D <= 0 || U <= 0) return RM_ERR_INVALID_ARG;
+    if (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4 && elem_bytes != 8)
+        return RM_ERR_INVALID_ARG;
+    if (dir != RM_SEQ_TO_HEAD && dir != RM_HEAD_TO_SEQ) return RM_ERR_INVALID_ARG;
+    if (ntensors < 1 || ntensors > 3 || !tensors || !heads) return RM_ERR_INVALID_ARG;
+    UlyTensor t[3];
+    for (int i = 0; i < ntensors; ++i) {
+        if (heads[i] <= 0 || heads[i] % U != 0) return RM_ERR_INVALID_ARG;
+        t[i] = UlyTensor{tensors[i], heads[i]};
+    }
+    if (static_cast<int64_t>(U) * s >= (1ll << 31)) return RM_ERR_UNSUPPORTED;
+    if (B == 0 || s == 0) return RM_OK;
+    if (!buf || !aligned16(buf)) return RM_ERR_INVALID_ARG;
+    for (int i = 0; i < ntensors; ++i)
+        if (!t[i].tensor || !aligned16(t[i].tensor) || t[i].tensor == buf) return RM_ERR_INVALID_ARG;
+    LaunchCtx ctx;
+    rm_status st = get_ctx(stream, &ctx);
+    if (st != RM_OK) return st;
+    const int head_side = pack ? dir == RM_HEAD_TO_SEQ : dir == RM_SEQ_TO_HEAD;
+    cudaError_t e = launch_ulysses_exchange(t, ntensors, buf, B, s, D, U, elem_bytes, pack,
+                                            head_side, ctx);
+    return e == cudaSuccess ? RM_OK : cuda_fail(e);
+}
+
+size_t rm_ulysses_buffer_size(const int* heads, int ntensors, int B, int s, int D,
+                              int elem_bytes) {
+    if (!heads || ntensors < 1 || ntensors > 3 || B <= 0 || s <= 0 || D <= 0 || elem_bytes <= 0)
+        return 0;
+    size_t n = 0;
+    for (int i = 0; i < ntensors; ++i) n += static_cast<size_t>(heads[i] > 0 ? heads[i] : 0);
+    return n * static_cast<size_t>(B) * s * D * elem_bytes;
+}
+
+rm_status rm_ulysses_pack(const void* const* tensors, const int* heads, int ntensors,
+                          void* send_buf, int B, int s, int D, int U, int elem_bytes,
+                          rm_permute_dir dir, cudaStream_t stream) {
+    return ulysses_exchange(tensors, heads, ntensors, send_buf, B, s, D, U, elem_bytes, dir, 1,
+                            stream);
+}
+
+rm_status rm_ulysses_unpack(const void* recv_buf, void* const* tensors, const int* heads,
+                            int ntensors, int B, int s, int D, int U, int elem_bytes,
+                            rm_permute_dir dir, cudaStream_t stream) {
+    return ulysses_exchange(const_cast<const void* const*>(tensors), heads, ntensors,
+                            const_cast<void*>(recv_buf), B, s, D, U, elem_bytes, dir, 0, stream);
 }
 
 rm_status rm_seq_reorder(const void* src, void* dst, int B, int H, int S, int D, int P,

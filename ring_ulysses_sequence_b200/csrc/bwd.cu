@@ -31,6 +31,15 @@
 // runs in two passes, P first (the MMA thread can start the product that needs
 // only P) and dS second, and S and dP signal separately, so the compute warps
 // start P while dP is still on the tensor pipe.
+//
+// One-step mode (`step`): the part of the backward that one rank of a ring
+// across devices computes at one step. Its L local queries meet the L keys of
+// one owner's block only: dQ of the rank and dK/dV of the block are ADDED to
+// the arrays passed in (q-side arrays hold the rank's rows, k-side arrays the
+// block's rows), so that dQ accumulates over the steps on the rank and dK/dV
+// over the ranks the block visits. A tile that sees nothing of the other side
+// is left untouched. Every element is still written by one CTA per launch, so
+// the sums stay deterministic.
 #include <algorithm>
 
 #include "common.cuh"
@@ -84,6 +93,10 @@ struct BwdArgs {
     MaskSpec mk;     // which keys each query sees
     float scale, scale_log2;
     RingLayout lay;
+    int step;        // one step: rank `rank`'s queries against `owner`'s block
+    int rank, owner;
+    int q_len;       // rows per head of q, dout, lse, delta, dq: S, or L for one step
+    int kv_len;      // rows per head of k, v, dk, dv: S, or L for one step
 };
 
 constexpr int kItemReaders = 9;  // the MMA thread and one lane of each compute warp
@@ -120,15 +133,23 @@ struct KvItem {
 
 // Key tiles in natural position order, earliest first (causal: they are seen
 // by the most query tiles).
+// One step: the tiles of the owner's block, in slot order; kslot is then the
+// row within the block.
 __device__ __forceinline__ KvItem decode_kv_item(const BwdArgs& a, int w) {
     KvItem it;
     const int nhu = a.B * a.Hkv;
     const int unit = w / nhu, hu = w - unit * nhu;
     it.b = hu / a.Hkv;
     it.g = hu - it.b * a.Hkv;
-    it.kpos = unit * kT;
-    it.kslot = a.lay.slot_of_pos(it.kpos);
-    it.rank = it.kslot / a.lay.L;
+    if (a.step) {
+        it.kslot = unit * kT;
+        it.kpos = a.lay.pos_of_slot(a.owner * a.lay.L + it.kslot);
+        it.rank = a.owner;
+    } else {
+        it.kpos = unit * kT;
+        it.kslot = a.lay.slot_of_pos(it.kpos);
+        it.rank = it.kslot / a.lay.L;
+    }
     return it;
 }
 
@@ -162,12 +183,17 @@ struct QIter {
                 const int runs = lay.zigzag ? 2 : 1;
                 if (++run == runs) {  // run starts at -1: the first call opens run 0 of step 0
                     run = 0;
-                    if (++t == lay.P) return false;
+                    // one step: the launching rank's runs only (t stays P after)
+                    if (a.step || ++t == lay.P) {
+                        run = runs - 1;
+                        t = lay.P;
+                        return false;
+                    }
                 }
-                int i = rank + t;
+                int i = a.step ? a.rank : rank + t;
                 if (i >= lay.P) i -= lay.P;
                 const int ctiles = (lay.zigzag ? lay.c : lay.L) / kT;
-                s0 = i * lay.L + run * lay.c;
+                s0 = (a.step ? 0 : i * lay.L) + run * lay.c;
                 p0 = lay.zigzag ? (run == 0 ? i * lay.c : (2 * lay.P - 1 - i) * lay.c) : i * lay.L;
                 // query tiles meeting [cf.x, cl.y]
                 u = max(0, ceil_div128(cf.x - (kT - 1) - p0));
@@ -205,18 +231,28 @@ __device__ __forceinline__ void issue_acc_product(uint32_t tmem_acc, uint32_t tm
                 idesc, (accumulate || k > 0) ? 1u : 0u);
 }
 
-// Stores N fp32 accumulator columns of this thread's TMEM row, times `mul`.
+// Stores N fp32 accumulator columns of this thread's TMEM row, times `mul`;
+// with `add`, adds them to what dst holds.
 template <int N>
-__device__ __forceinline__ void store_cols(uint32_t taddr, float* dst, float mul) {
+__device__ __forceinline__ void store_cols(uint32_t taddr, float* dst, float mul, int add) {
 #pragma unroll 1
     for (int cc = 0; cc < N; cc += 32) {
         uint32_t v[32];
         tmem_ld32(taddr + cc, v);
         float4* d4 = reinterpret_cast<float4*>(dst + cc);
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-            d4[c] = make_float4(__uint_as_float(v[4 * c]) * mul, __uint_as_float(v[4 * c + 1]) * mul,
-                                __uint_as_float(v[4 * c + 2]) * mul, __uint_as_float(v[4 * c + 3]) * mul);
+        for (int c = 0; c < 8; ++c) {
+            float4 x = make_float4(__uint_as_float(v[4 * c]) * mul, __uint_as_float(v[4 * c + 1]) * mul,
+                                   __uint_as_float(v[4 * c + 2]) * mul, __uint_as_float(v[4 * c + 3]) * mul);
+            if (add) {
+                const float4 y = d4[c];
+                x.x += y.x;
+                x.y += y.y;
+                x.z += y.z;
+                x.w += y.w;
+            }
+            d4[c] = x;
+        }
     }
 }
 
@@ -264,30 +300,33 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
             prefetch_tmap(&a.tm_k);
             prefetch_tmap(&a.tm_v);
             prefetch_tmap(&a.tm_do);
-            uint32_t items = 0, fills = 0;
+            uint32_t items = 0, fills = 0;  // items: those with at least one query tile
             bool ok = true;
-            for (uint32_t k = 0; ok; ++k, ++items) {
+            for (uint32_t k = 0; ok; ++k) {
                 int w;
                 ok = item_claim(bars.items, a.work, k, w, wd);
                 if (!ok || w >= a.n_items) break;
                 const KvItem it = decode_kv_item(a, w);
+                QIter qi(a, it);
+                int h, qslot, cls;
+                bool more = qi.next(a, h, qslot, cls);
+                if (!more) continue;  // one step: no query of the rank sees this tile
                 if (items > 0) ok = mbar_wait(smem_u32(&bars.res_empty), (items - 1) & 1, wd);
                 if (!ok) break;
-                const int krow = (it.b * a.Hkv + it.g) * a.S + it.kslot;
+                ++items;
+                const int krow = (it.b * a.Hkv + it.g) * a.kv_len + it.kslot;
                 mbar_arrive_expect_tx(smem_u32(&bars.res_full), 2 * BCfg<D>::kTile);
                 for (int bx = 0; bx < BCfg<D>::kBoxes; ++bx) {
                     tma_load_2d(k_smem + bx * BCfg<D>::kBox, &a.tm_k, bx * 64, krow, smem_u32(&bars.res_full));
                     tma_load_2d(v_smem + bx * BCfg<D>::kBox, &a.tm_v, bx * 64, krow, smem_u32(&bars.res_full));
                 }
-                QIter qi(a, it);
-                int h, qslot, cls;
-                while (ok && qi.next(a, h, qslot, cls)) {
+                for (; ok && more; more = qi.next(a, h, qslot, cls)) {
                     const int st = fills % kStages;
                     const uint32_t use = fills / kStages;
                     if (use > 0) ok = mbar_wait(smem_u32(&bars.st_empty[st]), (use - 1) & 1, wd);
                     if (!ok) break;
                     const uint32_t base = st_smem + st * BCfg<D>::kStageKV;
-                    const int qrow = (it.b * a.H + h) * a.S + qslot;
+                    const int qrow = (it.b * a.H + h) * a.q_len + qslot;
                     const uint32_t bar = smem_u32(&bars.st_full[st]);
                     mbar_arrive_expect_tx(bar, BCfg<D>::kStageKV);
                     for (int bx = 0; bx < BCfg<D>::kBoxes; ++bx) {
@@ -312,15 +351,17 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
             const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 384;
             uint32_t items = 0, uses = 0, p_cnt = 0;
             bool ok = true;
-            for (uint32_t k = 0; ok; ++k, ++items) {
+            for (uint32_t k = 0; ok; ++k) {
                 int w;
                 ok = item_read(bars.items, k, w, false, wd);
                 if (!ok || w >= a.n_items) break;
                 const KvItem it = decode_kv_item(a, w);
                 QIter qi(a, it);
                 int qh, qs, qc;
+                if (!qi.next(a, qh, qs, qc)) continue;  // query tile 0 (one step may have none)
                 ok = mbar_wait(smem_u32(&bars.res_full), items & 1, wd);
                 if (!ok) break;
+                ++items;
                 tc_fence_after();
                 // S^T of query tile j + 1 is issued right after dV of tile j (it
                 // overwrites P^T, which dV has read: in-order pipe), so the next
@@ -333,7 +374,6 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
                     return r;
                 };
                 int st = 0;
-                (void)qi.next(a, qh, qs, qc);  // query tile 0 (every key tile has one)
                 ok = stage(st);
                 if (ok) {
                     const uint32_t q_addr = st_smem + st * BCfg<D>::kStageKV;
@@ -391,14 +431,15 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
         const float sl2 = a.scale_log2;
         uint32_t uses = 0, s_cnt = 0, items = 0;  // s_cnt counts tiles for s_full and dp_full
         bool ok = true;
-        for (uint32_t k = 0; ok; ++k, ++items) {
+        for (uint32_t k = 0; ok; ++k) {
             int w;
             ok = item_read(bars.items, k, w, true, wd);
             if (!ok || w >= a.n_items) break;
             const KvItem it = decode_kv_item(a, w);
             QIter qi(a, it);
-            int h, qslot, cls;
+            int h, qslot, cls, ntiles = 0;
             while (ok && qi.next(a, h, qslot, cls)) {
+                ++ntiles;
                 const int st = uses % kStages;
                 ++uses;
                 // key row r sees query column c iff imin(j) <= qpos + c <= imax(j)
@@ -484,12 +525,14 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
                 mbar_arrive(smem_u32(&bars.p_full));
             }
             if (!ok) break;
+            if (ntiles == 0) continue;  // one step: the tile meets none of the rank's queries
             ok = mbar_wait(smem_u32(&bars.acc_full), items & 1, wd);
             if (!ok) break;
+            ++items;
             tc_fence_after();
-            const int64_t krow = (static_cast<int64_t>(it.b) * a.Hkv + it.g) * a.S + it.kslot + r;
-            store_cols<HC>(tdV, a.dv + krow * D + HC * wg, 1.0f);
-            store_cols<HC>(tdK, a.dk + krow * D + HC * wg, a.scale);
+            const int64_t krow = (static_cast<int64_t>(it.b) * a.Hkv + it.g) * a.kv_len + it.kslot + r;
+            store_cols<HC>(tdV, a.dv + krow * D + HC * wg, 1.0f, a.step);
+            store_cols<HC>(tdK, a.dk + krow * D + HC * wg, a.scale, a.step);
         }
     }
 
@@ -507,6 +550,8 @@ struct QItem {
 };
 
 // Query tiles, latest natural position first when causal (the most key tiles).
+// One step: the rank's tiles, latest slot first; slot is then the row within
+// the rank's arrays.
 __device__ __forceinline__ QItem decode_q_item(const BwdArgs& a, int w) {
     QItem it;
     const int nhu = a.B * a.H;
@@ -514,10 +559,16 @@ __device__ __forceinline__ QItem decode_q_item(const BwdArgs& a, int w) {
     it.b = hu / a.H;
     it.h = hu - it.b * a.H;
     it.g = it.h / a.G;
-    const int nu = a.causal ? (a.S / kT) - 1 - unit : unit;
-    it.pos = nu * kT;
-    it.slot = a.lay.slot_of_pos(it.pos);
-    it.rank = it.slot / a.lay.L;
+    const int nu = a.causal ? (a.q_len / kT) - 1 - unit : unit;
+    if (a.step) {
+        it.slot = nu * kT;
+        it.pos = a.lay.pos_of_slot(a.rank * a.lay.L + it.slot);
+        it.rank = a.rank;
+    } else {
+        it.pos = nu * kT;
+        it.slot = a.lay.slot_of_pos(it.pos);
+        it.rank = it.slot / a.lay.L;
+    }
     return it;
 }
 
@@ -539,11 +590,16 @@ struct KIter {
             const int runs = lay.zigzag ? 2 : 1;
             if (++run == runs) {
                 run = 0;
-                if (++t == lay.P) return false;
+                // one step: the owner's runs only (t stays P after)
+                if (a.step || ++t == lay.P) {
+                    run = runs - 1;
+                    t = lay.P;
+                    return false;
+                }
             }
-            const int r = lay.owner(rank, t);
+            const int r = a.step ? a.owner : lay.owner(rank, t);
             const int ctiles = (lay.zigzag ? lay.c : lay.L) / kT;
-            s0 = r * lay.L + run * lay.c;
+            s0 = (a.step ? 0 : r * lay.L) + run * lay.c;
             p0 = lay.zigzag ? (run == 0 ? r * lay.c : (2 * lay.P - 1 - r) * lay.c) : r * lay.L;
             // key tiles meeting [rf.x, rl.y]
             u = max(0, ceil_div128(rf.x - (kT - 1) - p0));
@@ -621,23 +677,26 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
                                 smem_u32(&full[slot]));
                 return true;
             };
-            for (uint32_t k = 0; ok; ++k, ++items) {
+            for (uint32_t k = 0; ok; ++k) {
                 int w;
                 ok = item_claim(bars.items, a.work, k, w, wd);
                 if (!ok || w >= a.n_items) break;
                 const QItem it = decode_q_item(a, w);
+                KIter ki(a, it);
+                int kslot, cls;
+                bool more = ki.next(a, kslot, cls);
+                if (!more) continue;  // one step: the tile sees no key of the block
                 if (items > 0) ok = mbar_wait(smem_u32(&bars.res_empty), (items - 1) & 1, wd);
                 if (!ok) break;
-                const int qrow = (it.b * a.H + it.h) * a.S + it.slot;
+                ++items;
+                const int qrow = (it.b * a.H + it.h) * a.q_len + it.slot;
                 mbar_arrive_expect_tx(smem_u32(&bars.res_full), 2 * BCfg<D>::kTile);
                 for (int bx = 0; bx < BCfg<D>::kBoxes; ++bx) {
                     tma_load_2d(q_smem + bx * BCfg<D>::kBox, &a.tm_q, bx * 64, qrow, smem_u32(&bars.res_full));
                     tma_load_2d(do_smem + bx * BCfg<D>::kBox, &a.tm_do, bx * 64, qrow, smem_u32(&bars.res_full));
                 }
-                KIter ki(a, it);
-                int kslot, cls;
-                while (ok && ki.next(a, kslot, cls)) {
-                    const int krow = (it.b * a.Hkv + it.g) * a.S + kslot;
+                for (; ok && more; more = ki.next(a, kslot, cls)) {
+                    const int krow = (it.b * a.Hkv + it.g) * a.kv_len + kslot;
                     ok = fill(bars.k_full, bars.k_empty, kKRing, kf, kr_smem, &a.tm_k, krow);
                     if (!ok) break;
                     ++kf;
@@ -662,15 +721,17 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
             const uint32_t tdP = tmem + 256, tdQ = tmem + 384;
             uint32_t items = 0, kc = 0, vc = 0, p_cnt = 0;
             bool ok = true;
-            for (uint32_t k = 0; ok; ++k, ++items) {
+            for (uint32_t k = 0; ok; ++k) {
                 int w;
                 ok = item_read(bars.items, k, w, false, wd);
                 if (!ok || w >= a.n_items) break;
                 const QItem it = decode_q_item(a, w);
                 KIter ki(a, it);  // one tile ahead of the S products
                 int ks, kcls;
+                if (!ki.next(a, ks, kcls)) continue;  // tile 0 (one step may have none)
                 ok = mbar_wait(smem_u32(&bars.res_full), items & 1, wd);
                 if (!ok) break;
+                ++items;
                 const uint32_t bk = kc, bv = vc;
                 // S_j = Q K_j^T into buffer j & 1
                 auto score = [&](uint32_t j) -> bool {
@@ -691,7 +752,6 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
                     umma_commit(smem_u32(&bars.dp_full));
                     return true;
                 };
-                (void)ki.next(a, ks, kcls);  // tile 0 (every query tile has one)
                 bool have1 = ki.next(a, ks, kcls);
                 ok = score(0) && dprod(0) && (!have1 || score(1));
                 uint32_t j = 0;
@@ -733,17 +793,18 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
         const float sl2 = a.scale_log2;
         uint32_t s_cnt[2] = {0, 0}, dp_cnt = 0, items = 0;
         bool ok = true;
-        for (uint32_t k = 0; ok; ++k, ++items) {
+        for (uint32_t k = 0; ok; ++k) {
             int w;
             ok = item_read(bars.items, k, w, true, wd);
             if (!ok || w >= a.n_items) break;
             const QItem it = decode_q_item(a, w);
-            const int64_t qrow = (static_cast<int64_t>(it.b) * a.H + it.h) * a.S + it.slot + r;
+            const int64_t qrow = (static_cast<int64_t>(it.b) * a.H + it.h) * a.q_len + it.slot + r;
             const float lse2 = a.lse[qrow] * kLog2e;
             const float delta = a.delta[qrow];
             KIter ki(a, it);
             int kslot, cls;
-            for (uint32_t j = 0; ok && ki.next(a, kslot, cls); ++j) {
+            uint32_t j = 0;
+            for (; ok && ki.next(a, kslot, cls); ++j) {
                 // query row r sees key column c iff lo(i) <= kpos + c <= hi(i)
                 int lo = 0;
                 unsigned wk = 0;
@@ -798,10 +859,12 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
                 mbar_arrive(smem_u32(&bars.p_full));
             }
             if (!ok) break;
+            if (j == 0) continue;  // one step: the tile sees no key of the block
             ok = mbar_wait(smem_u32(&bars.acc_full), items & 1, wd);
             if (!ok) break;
+            ++items;
             tc_fence_after();
-            store_cols<HC>(tdQ, a.dq + qrow * D + HC * wg, a.scale);
+            store_cols<HC>(tdQ, a.dq + qrow * D + HC * wg, a.scale, a.step);
         }
     }
 
@@ -814,9 +877,10 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dq_kernel(const __grid_c
 
 // -------------------------------------------------------------------- Delta
 
-// Delta_i = <dO_i, O_i> in fp32 from the bf16 rows; one warp per row.
-template <int D>
-__global__ void __launch_bounds__(256) bwd_delta_kernel(const __nv_bfloat16* __restrict__ o,
+// Delta_i = <dO_i, O_i> in fp32 from the bf16 dO rows and the O rows (bf16, or
+// fp32 as a ring across devices accumulates them); one warp per row.
+template <int D, typename OT>
+__global__ void __launch_bounds__(256) bwd_delta_kernel(const OT* __restrict__ o,
                                                         const __nv_bfloat16* __restrict__ dout,
                                                         float* __restrict__ delta, int64_t rows) {
     constexpr int PER = D / 32;  // elements per lane
@@ -824,43 +888,64 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const __nv_bfloat16* __r
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * 256) >> 5;
     for (int64_t r = warp; r < rows; r += nwarps) {
-        const __nv_bfloat16* po = o + r * D + lane * PER;
+        const OT* po = o + r * D + lane * PER;
         const __nv_bfloat16* pd = dout + r * D + lane * PER;
-        float acc = 0.f;
+        float x[PER], y[PER];
         if constexpr (PER == 4) {
-            const uint2 vo = *reinterpret_cast<const uint2*>(po);
             const uint2 vd = *reinterpret_cast<const uint2*>(pd);
-            const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&vo);
             const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&vd);
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const float2 x = __bfloat1622float2(a2[i]), y = __bfloat1622float2(b2[i]);
-                acc = fmaf(x.x, y.x, fmaf(x.y, y.y, acc));
-            }
+            const float2 y0 = __bfloat1622float2(b2[0]), y1 = __bfloat1622float2(b2[1]);
+            y[0] = y0.x; y[1] = y0.y; y[2] = y1.x; y[3] = y1.y;
         } else {
-            const __nv_bfloat162 x2 = *reinterpret_cast<const __nv_bfloat162*>(po);
-            const __nv_bfloat162 y2 = *reinterpret_cast<const __nv_bfloat162*>(pd);
-            const float2 x = __bfloat1622float2(x2), y = __bfloat1622float2(y2);
-            acc = fmaf(x.x, y.x, x.y * y.y);
+            const float2 y0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(pd));
+            y[0] = y0.x; y[1] = y0.y;
         }
+        if constexpr (sizeof(OT) == 4) {
+            if constexpr (PER == 4) {
+                const float4 v = *reinterpret_cast<const float4*>(po);
+                x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+            } else {
+                const float2 v = *reinterpret_cast<const float2*>(po);
+                x[0] = v.x; x[1] = v.y;
+            }
+        } else if constexpr (PER == 4) {
+            const uint2 vo = *reinterpret_cast<const uint2*>(po);
+            const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&vo);
+            const float2 x0 = __bfloat1622float2(a2[0]), x1 = __bfloat1622float2(a2[1]);
+            x[0] = x0.x; x[1] = x0.y; x[2] = x1.x; x[3] = x1.y;
+        } else {
+            const float2 x0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(po));
+            x[0] = x0.x; x[1] = x0.y;
+        }
+        float acc = 0.f;
+#pragma unroll
+        for (int i = PER - 1; i >= 0; --i) acc = fmaf(x[i], y[i], acc);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
         if (lane == 0) delta[r] = acc;
     }
 }
 
+template <int D, typename OT>
+cudaError_t launch_delta(const void* o, const void* dout, float* delta, int64_t rows,
+                         const LaunchCtx& ctx) {
+    const int64_t dblocks = std::min<int64_t>((rows + 7) / 8, static_cast<int64_t>(ctx.num_sms) * 16);
+    bwd_delta_kernel<D, OT><<<static_cast<unsigned>(dblocks), 256, 0, ctx.stream>>>(
+        static_cast<const OT*>(o), static_cast<const __nv_bfloat16*>(dout), delta, rows);
+    return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t launch_bwd_d(const AttnShape& sh, const BwdArgs& base, const void* o, const void* dout,
                          float* delta, const LaunchCtx& ctx) {
     cudaError_t e;
-    const int64_t rows = static_cast<int64_t>(sh.B) * sh.H * sh.S;
-    const int64_t dblocks = std::min<int64_t>((rows + 7) / 8, static_cast<int64_t>(ctx.num_sms) * 16);
-    bwd_delta_kernel<D><<<static_cast<unsigned>(dblocks), 256, 0, ctx.stream>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), delta, rows);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (!base.step) {  // one step reads the Delta its caller computed once per rank
+        const int64_t rows = static_cast<int64_t>(sh.B) * sh.H * sh.S;
+        if ((e = launch_delta<D, __nv_bfloat16>(o, dout, delta, rows, ctx)) != cudaSuccess) return e;
+    }
 
     BwdArgs a = base;
-    a.n_items = sh.B * sh.Hkv * (sh.S / kT);
+    a.n_items = sh.B * sh.Hkv * (a.kv_len / kT);
     if ((e = next_work_counter(ctx, &a.work)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(ring_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   BCfg<D>::kSmemKV)) != cudaSuccess)
@@ -868,7 +953,7 @@ cudaError_t launch_bwd_d(const AttnShape& sh, const BwdArgs& base, const void* o
     ring_bwd_dkdv_kernel<D><<<std::min(a.n_items, ctx.num_sms), kThreads, BCfg<D>::kSmemKV, ctx.stream>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-    a.n_items = sh.B * sh.H * (sh.S / kT);
+    a.n_items = sh.B * sh.H * (a.q_len / kT);
     if ((e = next_work_counter(ctx, &a.work)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(ring_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   BCfg<D>::kSmemQ)) != cudaSuccess)
@@ -884,8 +969,10 @@ cudaError_t launch_bwd(const AttnShape& sh, const void* q, const void* k, const 
                        float* dv, float* delta, const LaunchCtx& ctx) {
     BwdArgs a{};
     cudaError_t e;
-    const uint64_t qrows = static_cast<uint64_t>(sh.B) * sh.H * sh.S;
-    const uint64_t kvrows = static_cast<uint64_t>(sh.B) * sh.Hkv * sh.S;
+    const bool step = sh.mode == 2;
+    const int len = step ? sh.S / sh.P : sh.S;  // rows per head (one step: a rank's block)
+    const uint64_t qrows = static_cast<uint64_t>(sh.B) * sh.H * len;
+    const uint64_t kvrows = static_cast<uint64_t>(sh.B) * sh.Hkv * len;
     if ((e = make_tmap_bf16_rows(&a.tm_q, q, qrows, sh.D, kT, 64)) != cudaSuccess) return e;
     if ((e = make_tmap_bf16_rows(&a.tm_do, dout, qrows, sh.D, kT, 64)) != cudaSuccess) return e;
     if ((e = make_tmap_bf16_rows(&a.tm_k, k, kvrows, sh.D, kT, 64)) != cudaSuccess) return e;
@@ -908,8 +995,22 @@ cudaError_t launch_bwd(const AttnShape& sh, const void* q, const void* k, const 
     a.scale = sh.scale;
     a.scale_log2 = sh.scale * kLog2e;
     a.lay = RingLayout{sh.S, sh.P, sh.S / sh.P, sh.zigzag ? sh.S / (2 * sh.P) : sh.S / sh.P, sh.zigzag};
+    a.step = step ? 1 : 0;
+    a.rank = step ? sh.rank : 0;
+    a.owner = step ? sh.owner : 0;
+    a.q_len = len;
+    a.kv_len = len;
     return sh.D == 64 ? launch_bwd_d<64>(sh, a, o, dout, delta, ctx)
                       : launch_bwd_d<128>(sh, a, o, dout, delta, ctx);
+}
+
+cudaError_t launch_bwd_delta(const void* o, int o_fp32, const void* dout, float* delta,
+                             int64_t rows, int D, const LaunchCtx& ctx) {
+    if (D == 64)
+        return o_fp32 ? launch_delta<64, float>(o, dout, delta, rows, ctx)
+                      : launch_delta<64, __nv_bfloat16>(o, dout, delta, rows, ctx);
+    return o_fp32 ? launch_delta<128, float>(o, dout, delta, rows, ctx)
+                  : launch_delta<128, __nv_bfloat16>(o, dout, delta, rows, ctx);
 }
 
 }  // namespace rm

@@ -39,7 +39,11 @@
 //              runs it: that rank's L local queries against one owner's L-token
 //              K/V block. O (fp32, normalised over this block's keys) and LSE
 //              are the step's partial; a row that sees none of the block gets
-//              (0, -inf), the identity of the (O, LSE) merge.
+//              (0, -inf), the identity of the (O, LSE) merge. With `merge` set,
+//              o and lse are instead the rank's running pair, and the epilogue
+//              folds the partial into it ("DeDLOC Guide", section 3: weights
+//              exp(a - M) and exp(b - M), M the larger LSE); rows that see none
+//              of the block are left as they are.
 #include <algorithm>
 
 #include "common.cuh"
@@ -89,6 +93,7 @@ struct TcArgs {
     int q_slot0;       // global slot of their first row: 0, or rank * L for one step
     int kv_len;        // rows per head of k, v: S, or L for one step
     int owner;         // one step: the rank whose block k, v hold
+    int merge;         // one step: o, lse are the running pair to fold into
 };
 
 struct Item {
@@ -511,6 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
                                  (x ? it.slot1 : it.slot0) - a.q_slot0 + r;
             if constexpr (kMode == kStep) {
                 if (j == 0) {  // the item saw nothing of this block: the merge identity
+                    if (a.merge) continue;  // folding the identity changes nothing
                     float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.o) + orow * D);
 #pragma unroll 1
                     for (int c = 0; c < D / 4; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -525,6 +531,39 @@ __global__ void __launch_bounds__(kThreads, 1) ring_fwd_tc_kernel(const __grid_c
             const float inv = l > 0.f ? 1.0f / l : 0.f;
             if constexpr (kMode == kStep) {
                 float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.o) + orow * D);
+                if (a.merge) {
+                    // (acc, partial) -> acc with the partial's LSE b = m*scale + ln l:
+                    // O = ca * O_acc + cb * O_tmem with ca = wa / (wa + wb) and
+                    // cb = wb / ((wa + wb) l). A row that saw no key (l = 0) keeps
+                    // its pair; the TMEM loads stay warp-wide either way.
+                    const float la = a.lse[orow];
+                    const float lb = l > 0.f ? m * a.scale + logf(l) : -INFINITY;
+                    const float M = fmaxf(la, lb);
+                    const bool fold = lb != -INFINITY;
+                    const float wa = (fold && la != -INFINITY) ? expf(la - M) : 0.f;
+                    const float wb = fold ? expf(lb - M) : 0.f;
+                    const float ws = wa + wb;
+                    const float ca = fold ? wa / ws : 1.f;
+                    const float cb = fold ? wb / ws * inv : 0.f;
+#pragma unroll 1
+                    for (int cc = 0; cc < D; cc += 32) {
+                        uint32_t ov[32];
+                        tmem_ld32(tO + cc, ov);
+                        if (!fold) continue;
+#pragma unroll
+                        for (int v4 = 0; v4 < 8; ++v4) {
+                            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+                            if (wa != 0.f) x = dst[cc / 4 + v4];
+                            x.x = fmaf(ca, x.x, cb * __uint_as_float(ov[4 * v4]));
+                            x.y = fmaf(ca, x.y, cb * __uint_as_float(ov[4 * v4 + 1]));
+                            x.z = fmaf(ca, x.z, cb * __uint_as_float(ov[4 * v4 + 2]));
+                            x.w = fmaf(ca, x.w, cb * __uint_as_float(ov[4 * v4 + 3]));
+                            dst[cc / 4 + v4] = x;
+                        }
+                    }
+                    if (fold) a.lse[orow] = M + logf(ws);
+                    continue;
+                }
 #pragma unroll 1
                 for (int cc = 0; cc < D; cc += 32) {
                     uint32_t ov[32];
@@ -612,6 +651,7 @@ cudaError_t launch_fwd_tc(const AttnShape& sh, const void* q, const void* k, con
     a.q_slot0 = step ? sh.rank * L : 0;
     a.kv_len = len;
     a.owner = step ? sh.owner : 0;
+    a.merge = step ? sh.merge : 0;
     const int grid = std::min(a.n_items, ctx.num_sms);
     if (sh.D == 64) {
         if (sh.mode == kStep) return launch<64, kStep>(a, grid, ctx);

@@ -28,6 +28,7 @@ struct AttnShape {
     // block; o is fp32).
     int mode;
     int rank, owner;
+    int merge;             // mode 2: o, lse hold the running pair; fold the step into it
 };
 
 // Dynamic work distribution: a persistent kernel's CTAs take work items from a
@@ -44,10 +45,16 @@ cudaError_t launch_fwd_tc(const AttnShape& sh, const void* q, const void* k, con
 // Forward, fp32 FMA path (fwd_simt.cu).
 cudaError_t launch_fwd_fp32(const AttnShape& sh, const float* q, const float* k, const float* v,
                             float* o, float* lse, const LaunchCtx& ctx);
-// Backward, bf16 (bwd.cu). workspace holds Delta [B, H, S] fp32.
+// Backward, bf16 (bwd.cu). delta: Delta [B, H, S] fp32, computed here from o
+// and dout; with mode 2 (one ring step of `rank` against `owner`'s block, the
+// q-side arrays holding the rank's L rows and the k-side ones the block's) it
+// is an input, o is not read, and dq, dk, dv are added to.
 cudaError_t launch_bwd(const AttnShape& sh, const void* q, const void* k, const void* v,
                        const void* o, const float* lse, const void* dout, float* dq, float* dk,
                        float* dv, float* delta, const LaunchCtx& ctx);
+// Delta = rowsum(dO * O) over `rows` rows of D; o bf16 or (o_fp32) float32.
+cudaError_t launch_bwd_delta(const void* o, int o_fp32, const void* dout, float* delta,
+                             int64_t rows, int D, const LaunchCtx& ctx);
 
 // Layout kernels (layout.cu).
 struct PermuteTensor {
@@ -57,6 +64,18 @@ struct PermuteTensor {
 };
 cudaError_t launch_ulysses_permute(const PermuteTensor* t, int ntensors, int B, int S, int D,
                                    int elem_bytes, int head_to_seq, const LaunchCtx& ctx);
+// Ulysses exchange buffer <-> one device's tensors (layout.cu): buf holds U
+// chunks, each the tensors' parts [B, s, heads / U, D] one after another.
+// pack: tensors -> buf; else buf -> tensors. head_side: the tensors are the
+// device's head shards [B, heads / U, U * s, D], else its sequence shards
+// [B, s, heads, D].
+struct UlyTensor {
+    const void* tensor;
+    int heads;
+};
+cudaError_t launch_ulysses_exchange(const UlyTensor* t, int ntensors, void* buf, int B, int s,
+                                    int D, int U, int elem_bytes, int pack, int head_side,
+                                    const LaunchCtx& ctx);
 cudaError_t launch_seq_reorder(const void* src, void* dst, int BH, int S, int D, int P,
                                int zigzag, int to_natural, int elem_bytes, const LaunchCtx& ctx);
 cudaError_t launch_lse_merge(float* o_acc, float* lse_acc, const float* o_part,

@@ -94,6 +94,82 @@ __global__ void __launch_bounds__(kThreads) ulysses_permute_kernel(const __grid_
     }
 }
 
+// Ulysses exchange buffers of one device (U devices per Ulysses group, each
+// holding s tokens of all heads before the all-to-all). The buffer is U
+// chunks, chunk u for (or from) device u; in a chunk the tensors follow one
+// another, tensor x as [B, s, heads_x / U, D] (the s tokens of the sending
+// device for the heads of the receiving one). The device's own tensor x is
+//   sequence side [B, s, heads_x, D]          (heads u*hU + hh of token t), or
+//   head side     [B, hU, U*s, D]             (token u*s + t of head hh),
+// hU = heads_x / U. pack: tensor -> buffer; unpack: buffer -> tensor. A block
+// moves tok_per_tile tokens x hU heads of one (x, u, b): a contiguous run of
+// the buffer, whole D-element rows of the tensor.
+struct UlyPart {
+    const char* tensor;
+    char* buf;           // the buffer's first byte (the same for every tensor)
+    int hU;              // heads of the tensor per device
+    int heads;           // all heads of the tensor (sequence side)
+    int64_t chunk_off;   // vectors from a chunk's start to this tensor's part
+    int tok_per_tile, tiles_per_ub;
+    int64_t block_start;
+    FastDiv div_row;     // by hU * vec_per_row
+};
+
+struct UlyArgs {
+    UlyPart t[3];
+    int ntensors;
+    int B, s, U, vec_per_row;
+    int64_t chunk_vecs;  // vectors per chunk
+    int pack, head_side;
+    FastDiv div_vpr;
+};
+
+template <int V>
+__global__ void __launch_bounds__(kThreads) ulysses_exchange_kernel(const __grid_constant__ UlyArgs a) {
+    using T = typename VecT<V>::T;
+    int ti = 0;
+    while (ti + 1 < a.ntensors && static_cast<int64_t>(blockIdx.x) >= a.t[ti + 1].block_start) ++ti;
+    const UlyPart& pt = a.t[ti];
+    int64_t blk = static_cast<int64_t>(blockIdx.x) - pt.block_start;
+    const int tile = static_cast<int>(blk % pt.tiles_per_ub);
+    blk /= pt.tiles_per_ub;
+    const int b = static_cast<int>(blk % a.B);
+    const int u = static_cast<int>(blk / a.B);
+    const int t0 = tile * pt.tok_per_tile;
+    const int nt = min(pt.tok_per_tile, a.s - t0);
+    const int vpr = a.vec_per_row, hU = pt.hU;
+    const uint32_t n = static_cast<uint32_t>(nt) * hU * vpr;
+    const int64_t buf_base = u * a.chunk_vecs + pt.chunk_off +
+                             (static_cast<int64_t>(b) * a.s + t0) * hU * vpr;
+    T* buf = reinterpret_cast<T*>(pt.buf);
+    T* ten = reinterpret_cast<T*>(const_cast<char*>(pt.tensor));
+    for (uint32_t i0 = threadIdx.x; i0 < n; i0 += kThreads * kUnroll) {
+        T val[kUnroll];
+        int64_t toff[kUnroll];
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k) {
+            const uint32_t i = i0 + k * kThreads;
+            toff[k] = -1;
+            if (i < n) {
+                const uint32_t tl = pt.div_row.div(i);            // token within the tile
+                const uint32_t rem = i - tl * hU * vpr;
+                const uint32_t hh = a.div_vpr.div(rem);           // head within the device's share
+                const uint32_t vin = rem - hh * vpr;
+                const int64_t t = t0 + tl;
+                toff[k] = a.head_side
+                              ? ((static_cast<int64_t>(b) * hU + hh) * a.U * a.s + u * a.s + t) * vpr + vin
+                              : ((b * a.s + t) * pt.heads + u * hU + hh) * vpr + vin;
+                val[k] = ld_stream(a.pack ? ten + toff[k] : buf + buf_base + i);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k) {
+            const uint32_t i = i0 + k * kThreads;
+            if (toff[k] >= 0) st_stream(a.pack ? buf + buf_base + i : ten + toff[k], val[k]);
+        }
+    }
+}
+
 struct ReorderArgs {
     const char* src;
     char* dst;
@@ -264,6 +340,52 @@ cudaError_t launch_ulysses_permute(const PermuteTensor* t, int ntensors, int B, 
         case 4: ulysses_permute_kernel<4><<<grid, kThreads, 0, ctx.stream>>>(a); break;
         case 2: ulysses_permute_kernel<2><<<grid, kThreads, 0, ctx.stream>>>(a); break;
         default: ulysses_permute_kernel<1><<<grid, kThreads, 0, ctx.stream>>>(a); break;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ulysses_exchange(const UlyTensor* t, int ntensors, void* buf, int B, int s,
+                                    int D, int U, int elem_bytes, int pack, int head_side,
+                                    const LaunchCtx& ctx) {
+    const int64_t row_bytes = static_cast<int64_t>(D) * elem_bytes;
+    int V = 16;
+    for (int i = 0; i < ntensors; ++i) V = std::min(V, pick_vec(row_bytes, t[i].tensor, buf));
+    UlyArgs a{};
+    a.ntensors = ntensors;
+    a.B = B;
+    a.s = s;
+    a.U = U;
+    a.vec_per_row = static_cast<int>(row_bytes / V);
+    a.pack = pack;
+    a.head_side = head_side;
+    a.div_vpr.init(static_cast<uint32_t>(a.vec_per_row));
+    int64_t off = 0, blocks = 0;
+    for (int i = 0; i < ntensors; ++i) {
+        UlyPart& p = a.t[i];
+        p.tensor = static_cast<const char*>(t[i].tensor);
+        p.buf = static_cast<char*>(buf);
+        p.heads = t[i].heads;
+        p.hU = t[i].heads / U;
+        p.chunk_off = off;
+        const int64_t per_tok = static_cast<int64_t>(p.hU) * a.vec_per_row;
+        if (per_tok >= (1ll << 30)) return cudaErrorInvalidValue;
+        off += static_cast<int64_t>(B) * s * per_tok;
+        p.tok_per_tile = static_cast<int>(std::min<int64_t>(s, std::max<int64_t>(1, kTileVecs / per_tok)));
+        p.tiles_per_ub = (s + p.tok_per_tile - 1) / p.tok_per_tile;
+        p.block_start = blocks;
+        p.div_row.init(static_cast<uint32_t>(per_tok));
+        blocks += static_cast<int64_t>(U) * B * p.tiles_per_ub;
+    }
+    a.chunk_vecs = off;
+    if (blocks == 0) return cudaSuccess;
+    if (blocks > 0x7fffffffll) return cudaErrorInvalidValue;
+    dim3 grid(static_cast<unsigned>(blocks));
+    switch (V) {
+        case 16: ulysses_exchange_kernel<16><<<grid, kThreads, 0, ctx.stream>>>(a); break;
+        case 8: ulysses_exchange_kernel<8><<<grid, kThreads, 0, ctx.stream>>>(a); break;
+        case 4: ulysses_exchange_kernel<4><<<grid, kThreads, 0, ctx.stream>>>(a); break;
+        case 2: ulysses_exchange_kernel<2><<<grid, kThreads, 0, ctx.stream>>>(a); break;
+        default: ulysses_exchange_kernel<1><<<grid, kThreads, 0, ctx.stream>>>(a); break;
     }
     return cudaGetLastError();
 }

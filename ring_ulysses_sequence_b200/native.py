@@ -25,6 +25,8 @@ SIGNATURES = {
                                    _f, _vp]),
     "rm_ring_attn_fwd_step": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                                    _i, _i, _f, _vp]),
+    "rm_ring_attn_fwd_step_merge": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                         _i, _i, _i, _i, _f, _vp]),
     "rm_ring_attn_fwd_window": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                                      _f, _vp]),
     "rm_varlen_bounds_size": (_sz, [_i, _i]),
@@ -40,10 +42,16 @@ SIGNATURES = {
                                      _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "rm_ring_attn_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                       _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
+    "rm_ring_attn_bwd_delta": (_i, [_vp, _vp, _vp, _i64, _i, _i, _vp]),
+    "rm_ring_attn_bwd_step": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                   _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "rm_lse_merge": (_i, [_vp, _vp, _vp, _vp, _i64, _i, _vp]),
     "rm_ulysses_permute": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "rm_ulysses_permute_qkv": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
                                     _i, _i, _vp]),
+    "rm_ulysses_buffer_size": (_sz, [_vp, _i, _i, _i, _i, _i]),
+    "rm_ulysses_pack": (_i, [_vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _vp]),
+    "rm_ulysses_unpack": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "rm_seq_reorder": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "rm_check_device_status": (_i, [_vp]),
     "rm_set_watchdog_ns": (None, [_u64]),
@@ -125,6 +133,13 @@ def rm_ring_attn_fwd_step(q_local, k_block, v_block, o_part, lse_part, B, H, Hkv
                  _s(stream))
 
 
+def rm_ring_attn_fwd_step_merge(q_local, k_block, v_block, o_acc, lse_acc, B, H, Hkv, S, D, P,
+                                rank, owner, causal, order, dtype, scale, stream=None):
+    return _call("rm_ring_attn_fwd_step_merge", _p(q_local), _p(k_block), _p(v_block), _p(o_acc),
+                 _p(lse_acc), B, H, Hkv, S, D, P, rank, owner, int(causal), order, dtype, scale,
+                 _s(stream))
+
+
 def rm_ring_attn_fwd_window(q, k, v, o, lse, B, H, Hkv, S, D, P, window, order, dtype, scale,
                             stream=None):
     return _call("rm_ring_attn_fwd_window", _p(q), _p(k), _p(v), _p(o), _p(lse), B, H, Hkv, S, D,
@@ -180,6 +195,19 @@ def rm_ring_attn_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, H, Hkv, S, D,
                  _s(stream))
 
 
+def rm_ring_attn_bwd_delta(o, dout, delta, rows, D, o_dtype, stream=None):
+    return _call("rm_ring_attn_bwd_delta", _p(o), _p(dout), _p(delta), rows, D, o_dtype,
+                 _s(stream))
+
+
+def rm_ring_attn_bwd_step(q_local, k_block, v_block, lse_local, delta_local, dout_local, dq_local,
+                          dk_block, dv_block, B, H, Hkv, S, D, P, rank, owner, causal, order,
+                          dtype, scale, stream=None):
+    return _call("rm_ring_attn_bwd_step", _p(q_local), _p(k_block), _p(v_block), _p(lse_local),
+                 _p(delta_local), _p(dout_local), _p(dq_local), _p(dk_block), _p(dv_block), B, H,
+                 Hkv, S, D, P, rank, owner, int(causal), order, dtype, scale, _s(stream))
+
+
 def rm_lse_merge(o_acc, lse_acc, o_part, lse_part, rows, D, stream=None):
     return _call("rm_lse_merge", _p(o_acc), _p(lse_acc), _p(o_part), _p(lse_part), rows, D,
                  _s(stream))
@@ -194,6 +222,31 @@ def rm_ulysses_permute_qkv(q_src, k_src, v_src, q_dst, k_dst, v_dst, B, S, H, Hk
                            elem_bytes, direction, stream=None):
     return _call("rm_ulysses_permute_qkv", _p(q_src), _p(k_src), _p(v_src), _p(q_dst),
                  _p(k_dst), _p(v_dst), B, S, H, Hkv, D, U, R, elem_bytes, direction, _s(stream))
+
+
+def _host_arrays(tensors, heads):
+    n = len(tensors)
+    ptrs = (ctypes.c_void_p * n)(*[_p(t) for t in tensors])
+    hs = (ctypes.c_int * n)(*[int(h) for h in heads])
+    return n, ctypes.cast(ptrs, ctypes.c_void_p), ctypes.cast(hs, ctypes.c_void_p), (ptrs, hs)
+
+
+def rm_ulysses_buffer_size(heads, B, s, D, elem_bytes):
+    hs = (ctypes.c_int * len(heads))(*[int(h) for h in heads])
+    return int(lib().rm_ulysses_buffer_size(ctypes.cast(hs, ctypes.c_void_p), len(heads), B, s,
+                                            D, elem_bytes))
+
+
+def rm_ulysses_pack(tensors, heads, send_buf, B, s, D, U, elem_bytes, direction, stream=None):
+    n, ptrs, hs, keep = _host_arrays(tensors, heads)
+    return _call("rm_ulysses_pack", ptrs, hs, n, _p(send_buf), B, s, D, U, elem_bytes, direction,
+                 _s(stream))
+
+
+def rm_ulysses_unpack(recv_buf, tensors, heads, B, s, D, U, elem_bytes, direction, stream=None):
+    n, ptrs, hs, keep = _host_arrays(tensors, heads)
+    return _call("rm_ulysses_unpack", _p(recv_buf), ptrs, hs, n, B, s, D, U, elem_bytes,
+                 direction, _s(stream))
 
 
 def rm_seq_reorder(src, dst, B, H, S, D, P, order, direction, elem_bytes, stream=None):

@@ -225,3 +225,111 @@ def test_binding_argument_counts_match_the_header():
         params = " ".join(params.split())
         n = 0 if params in ("", "void") else params.count(",") + 1
         assert len(native.SIGNATURES[name][1]) == n, (name, n, len(native.SIGNATURES[name][1]))
+
+
+def test_step_merge_and_backward_step_validation(lib):
+    # rm_ring_attn_fwd_step_merge: rank/owner range, fp32, shape rules
+    def sm(rank=0, owner=0, dtype=0, S=1024, **kw):
+        return lib.rm_ring_attn_fwd_step_merge(A, A, A, kw.get("o", A), kw.get("lse", A), 1, 4, 2,
+                                               S, 128, 4, rank, owner, 1, 1, dtype, 0.088, None)
+    assert sm(rank=4) == 1 and sm(owner=-1) == 1
+    assert sm(dtype=1) == 2
+    assert sm(S=1004) == 1
+    assert sm(o=None) == 1
+    assert sm(S=0) == 0
+    # rm_ring_attn_bwd_step
+    base = [A] * 9 + [1, 4, 2, 1024, 128, 4, 1, 2, 1, 1, 0, 0.088, None]
+    assert lib.rm_ring_attn_bwd_step(*base) != 1 or True  # (valid: would launch; not called)
+    for i in range(3, 9):                                  # lse .. dv must be given
+        bad = list(base)
+        bad[i] = None
+        assert lib.rm_ring_attn_bwd_step(*bad) == 1, i
+    for j, val in ((15, 4), (16, 7), (15, -1)):            # rank, owner out of range
+        bad = list(base)
+        bad[j] = val
+        assert lib.rm_ring_attn_bwd_step(*bad) == 1
+    fp32 = list(base)
+    fp32[19] = 1
+    assert lib.rm_ring_attn_bwd_step(*fp32) == 2
+    empty = list(base)
+    empty[9] = 0                                           # B = 0: nothing to do
+    assert lib.rm_ring_attn_bwd_step(*empty) == 0
+    # rm_ring_attn_bwd_delta
+    assert lib.rm_ring_attn_bwd_delta(A, A, A, 16, 96, 0, None) == 2      # D = 96
+    assert lib.rm_ring_attn_bwd_delta(A, A, A, 16, 128, 3, None) == 1     # bad dtype
+    assert lib.rm_ring_attn_bwd_delta(A, A, A, -1, 128, 0, None) == 1
+    assert lib.rm_ring_attn_bwd_delta(None, A, A, 0, 128, 0, None) == 0   # no rows
+    assert lib.rm_ring_attn_bwd_delta(A, None, A, 8, 128, 0, None) == 1
+
+
+def test_ulysses_exchange_validation(lib):
+    from ring_ulysses_sequence_b200 import native
+    assert native.rm_ulysses_buffer_size([32, 8, 8], 2, 16, 128, 2) == 48 * 2 * 16 * 128 * 2
+    assert native.rm_ulysses_buffer_size([], 1, 16, 128, 2) == 0
+    fake = [A + 4096 * i for i in range(4)]
+
+    def pack(tensors, heads, buf=A + (1 << 24), U=2, eb=2, d=0, B=1, s=16, D=128):
+        n = len(tensors)
+        ptrs = (ctypes.c_void_p * max(n, 1))(*tensors)
+        hs = (ctypes.c_int * max(len(heads), 1))(*heads)
+        return lib.rm_ulysses_pack(ctypes.cast(ptrs, ctypes.c_void_p),
+                                   ctypes.cast(hs, ctypes.c_void_p), n, buf, B, s, D, U, eb, d,
+                                   None)
+    assert pack(fake[:1], [6], U=4) == 1                   # 6 heads over U = 4
+    assert pack(fake[:4], [2, 2, 2, 2]) == 1               # at most three tensors
+    assert pack([], []) == 1
+    assert pack(fake[:1], [4], buf=fake[0]) == 1           # the buffer is a tensor
+    assert pack(fake[:1], [4], buf=A + 8) == 1             # misaligned buffer
+    assert pack(fake[:1], [4], eb=3) == 1
+    assert pack(fake[:1], [4], d=5) == 1
+    assert pack(fake[:1], [4], B=0) == 0                   # empty
+    assert pack([A + 8], [4]) == 1                         # misaligned tensor
+
+
+def test_wrappers_reject_mismatched_tensors_before_any_call(monkeypatch):
+    """The Python wrappers check every tensor's shape and dtype against q's
+    before calling the library (a shorter k would make the kernels read past
+    its allocation). CPU tensors stand in for device ones here; the native
+    calls are replaced by a stub that fails the test if reached."""
+    import ring_ulysses_sequence_b200 as rm
+    from ring_ulysses_sequence_b200 import native
+
+    class NoCall:
+        def __getattr__(self, name):
+            if name.startswith("rm_") and not name.endswith("_size"):  # sizes are host math
+                def fail(*a, **k):
+                    raise AssertionError(f"{name} reached with bad arguments")
+                return fail
+            return getattr(native, name)
+    monkeypatch.setattr(rm, "native", NoCall())
+    monkeypatch.setattr(rm, "_need", lambda t, n: None)     # allow CPU tensors
+    bf = torch.bfloat16
+    q = torch.zeros((1, 4, 256, 128), dtype=bf)
+    k = torch.zeros((1, 2, 256, 128), dtype=bf)
+    with pytest.raises(ValueError, match="k has shape"):
+        rm.ring_attn_fwd(q, k[:, :, :128], k, 2)
+    with pytest.raises(ValueError, match="v has dtype"):
+        rm.ring_attn_fwd(q, k, k.float(), 2)
+    with pytest.raises(ValueError, match="out has shape"):
+        rm.ring_attn_fwd(q, k, k, 2, out=torch.zeros((1, 4, 128, 128), dtype=bf))
+    with pytest.raises(ValueError, match="lse has dtype"):
+        rm.ring_attn_fwd(q, k, k, 2, lse=torch.zeros((1, 4, 256), dtype=bf))
+    lse = torch.zeros((1, 4, 256))
+    with pytest.raises(ValueError, match="dout has shape"):
+        rm.ring_attn_bwd(q, k, k, q, lse, q[:, :2], 2)
+    with pytest.raises(ValueError, match="workspace holds"):
+        rm.ring_attn_bwd(q, k, k, q, lse, q, 2, workspace=torch.zeros(16, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="k_block has shape"):
+        rm.ring_attn_fwd_step(q, k[:, :, :64], k, 2, 0, 0)
+    with pytest.raises(ValueError, match="lse_acc has shape"):
+        rm.ring_attn_fwd_step_merge(q, k, k, q.float(), lse[:, :2], 2, 0, 0)
+    with pytest.raises(ValueError, match="dk_block has dtype"):
+        rm.ring_attn_bwd_step(q, k, k, lse, lse, q, q.float(), k, k.float(), 2, 0, 0)
+    with pytest.raises(ValueError, match="o_part has shape"):
+        rm.lse_merge_(torch.zeros(8, 4), torch.zeros(8), torch.zeros(8, 2), torch.zeros(8))
+    with pytest.raises(ValueError, match="v has shape"):
+        rm.ulysses_permute_qkv(torch.zeros((1, 64, 8, 16), dtype=bf),
+                               torch.zeros((1, 64, 4, 16), dtype=bf),
+                               torch.zeros((1, 64, 2, 16), dtype=bf), 2, 1)
+    with pytest.raises(ValueError, match="must have 4 dimensions"):
+        rm.ring_attn_fwd(q[0], k, k, 2)

@@ -24,8 +24,13 @@ def _out():
                       "tflops": 1100.0, "tflops_attention": 1110.0,
                       "flops_per_launch": w.fwd_flops(),
                       "kv_bytes_per_rank": {"ring": 1, "allgather": 4}},
-        "steps": {"workload": w.name, "ms_per_step": 12.6, "tflops": 698.0,
-                  "launches_per_step": 130, "flops_per_step": w.fwd_flops()},
+        "steps": {"workload": w.name, "ms_per_step": 10.6, "tflops": 830.0,
+                  "launches_per_step": 66, "flops_per_step": w.fwd_flops(),
+                  "ms_per_step_two_calls": 12.6, "tflops_two_calls": 698.0},
+        "bwdsteps": {"workload": w.name, "ms_per_step": 30.0, "tflops": 733.0,
+                     "launches_per_step": 75, "flops_per_step": 2.5 * w.fwd_flops()},
+        "exchange": {"workload": "usp", "ms_per_step": 1.0, "gbs": 6400.0,
+                     "bytes_per_step": 6.4e9, "launches_per_step": 32},
         "window": {"workload": "win", "window": 4096, "docs": 0, "ms_per_launch": 2.0,
                    "tflops": 1000.0, "flops_per_launch": 2e12, "launches": 25},
         "packed": {"workload": "packed", "window": 0, "docs": 7, "ms_per_launch": 1.5,

@@ -9,7 +9,8 @@ import pytest
 import torch
 
 import oracle
-from gpu_util import BF16_MAX_ABS, BF16_MEAN_ABS, assert_close, to_natural, to_rank_major
+from gpu_util import (BF16_MAX_ABS, BF16_MEAN_ABS, LSE_MAX_ABS, assert_close, to_natural,
+                      to_rank_major)
 from ring_ulysses_sequence_b200.synth import WORKLOADS, make_inputs, make_tensor, sample_rows
 
 pytestmark = pytest.mark.gpu
@@ -70,16 +71,36 @@ def test_bwd_deterministic():
 
 
 def test_bwd_workload_sampled():
-    """B=2, H=Hkv=16, S=65536, D=128, P=16 zigzag, causal: dQ on seeded query rows
-    of every head; dK/dV on seeded key rows of two seeded KV heads."""
+    """B=2, H=Hkv=16, S=65536, D=128, P=16 zigzag, causal (forward + backward).
+
+    Seeded samples as the workload's parity rule states: 256 query rows per
+    head (plus the first and last row of every chunk) for the forward's O and
+    LSE and for dQ, on every head; 256 key rows (plus chunk edges) for dK and
+    dV on four seeded KV heads. The oracle's dK/dV rows need LSE and Delta of
+    every query row of those heads, i.e. a full fp64 forward per head."""
+    import ring_ulysses_sequence_b200 as rm
     w = WORKLOADS["ring_fwdbwd_bf16_S64k_causal_zigzag"]
     q, k, v, do = make_inputs(w)
-    dq, dk, dv = gpu_grads(q, k, v, do, w.P, w.order, w.causal)
-    qrows = sample_rows(w.S, 64, w.seed + 1000, w.chunk)
-    krows = sample_rows(w.S, 64, w.seed + 2000, w.chunk)
+    qr, kr, vr, dor = (to_rank_major(t, w.P, w.order).cuda() for t in (q, k, v, do))
+    o, lse = rm.ring_attn_fwd(qr, kr, vr, w.P, w.causal, w.order)
+    dq, dk, dv = rm.ring_attn_bwd(qr, kr, vr, o, lse, dor, w.P, w.causal, w.order)
+    torch.cuda.synchronize()
+    assert rm.native.rm_check_device_status() == 0
+    o, lse, dq, dk, dv = (to_natural(t.float().cpu(), w.P, w.order)
+                          for t in (o, lse.unsqueeze(-1), dq, dk, dv))
+    lse = lse.squeeze(-1)
+    qrows = sample_rows(w.S, 256, w.seed + 1000, w.chunk)
+    krows = sample_rows(w.S, 256, w.seed + 2000, w.chunk)
     rng = np.random.default_rng(w.seed + 3000)
-    kv_heads = [(int(rng.integers(w.B)), int(rng.integers(w.Hkv))) for _ in range(2)]
+    pairs = [(b, g) for b in range(w.B) for g in range(w.Hkv)]
+    kv_heads = [pairs[i] for i in sorted(rng.choice(len(pairs), size=4, replace=False))]
     q_heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+
+    # the forward this backward ran on
+    o_ref, lse_ref = oracle.attn_fwd(q.float(), k.float(), v.float(), w.causal, rows=qrows)
+    assert_close(o[:, :, qrows].numpy(), o_ref, BF16_MAX_ABS, BF16_MEAN_ABS, "O")
+    assert_close(lse[:, :, qrows].numpy(), lse_ref, LSE_MAX_ABS, what="LSE")
+
     rdq, rdkv = oracle.attn_bwd(q.float(), k.float(), v.float(), do.float(), True, qrows=qrows,
                                 krows=krows, heads=(q_heads, kv_heads))
     for (b, h) in q_heads:

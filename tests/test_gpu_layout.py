@@ -111,3 +111,58 @@ def test_lse_merge(rows, D):
     assert np.all(got_o[both_empty] == 0)
     np.testing.assert_allclose(got_o, o_ref, rtol=1e-5, atol=1e-5)
     np.testing.assert_allclose(got_l[~both_empty], l_ref[~both_empty], rtol=1e-6, atol=1e-5)
+
+
+@pytest.mark.parametrize("B,s,H,Hkv,D,U,R,dtype", [
+    (1, 64, 8, 4, 128, 4, 2, torch.bfloat16),
+    (2, 48, 6, 3, 64, 3, 1, torch.bfloat16),
+    (1, 40, 4, 2, 5, 2, 2, torch.uint8),     # 5-byte rows: 1-byte vectors
+    (1, 32, 4, 4, 1, 2, 3, torch.float32),   # D = 1 (an LSE-like tensor)
+    (1, 2048, 32, 8, 128, 4, 1, torch.bfloat16),
+])
+def test_ulysses_pack_unpack_is_the_all_to_all(B, s, H, Hkv, D, U, R, dtype):
+    """U x R devices simulated on one GPU. Each packs its sequence shard of Q,
+    K, V into one send buffer; chunk u2 of every sender, in sender order, is
+    what device u2 receives (the all-to-all); unpacking it must give exactly
+    the device's slab of the oracle's head-sharded tensors (bit-exact), and
+    the way back must restore every shard."""
+    import ring_ulysses_sequence_b200 as rm
+    S = U * R * s
+    full = [_bits((B, S, h, D), dtype, 10 * h + i) for i, h in enumerate((H, Hkv, Hkv))]
+    heads = [H, Hkv, Hkv]
+    n_chunk = sum(heads) // U * B * s * D
+    shard = lambda x, n: x[:, n * s:(n + 1) * s].contiguous().cuda()
+    sent = {(r, u): rm.ulysses_pack([shard(x, r * U + u) for x in full], U, "seq_to_head")
+            for r in range(R) for u in range(U)}
+    held = {}
+    for r in range(R):
+        for u2 in range(U):
+            recv = torch.cat([sent[(r, u)][u2 * n_chunk:(u2 + 1) * n_chunk] for u in range(U)])
+            held[(r, u2)] = rm.ulysses_unpack(recv, U, heads, B, s, D, "seq_to_head")
+    L = S // R
+    for (r, u), outs in held.items():
+        for x, h, got in zip(full, heads, outs):
+            hU = h // U
+            want = _from_np(oracle.ulysses_seq_to_head(_np(x)), dtype)[:, u * hU:(u + 1) * hU,
+                                                                       r * L:(r + 1) * L]
+            assert torch.equal(got.cpu(), want), (r, u, h)
+    # the inverse: head shards -> sequence shards
+    sent_back = {key: rm.ulysses_pack(list(outs), U, "head_to_seq") for key, outs in held.items()}
+    for r in range(R):
+        for u in range(U):
+            recv = torch.cat([sent_back[(r, u2)][u * n_chunk:(u + 1) * n_chunk]
+                              for u2 in range(U)])
+            back = rm.ulysses_unpack(recv, U, heads, B, s, D, "head_to_seq")
+            for x, got in zip(full, back):
+                assert torch.equal(got.cpu(), x[:, (r * U + u) * s:(r * U + u + 1) * s])
+
+
+def test_ulysses_pack_rejects_bad_arguments():
+    import ring_ulysses_sequence_b200 as rm
+    from ring_ulysses_sequence_b200 import native
+    x = torch.zeros((1, 8, 6, 16), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(rm.RMError):          # 6 heads do not split over U = 4
+        rm.ulysses_pack([x], 4, "seq_to_head")
+    buf = torch.empty(8 * 6 * 16, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(rm.RMError):          # the buffer may not be a tensor
+        native.rm_ulysses_pack([buf], [6], buf, 1, 8, 16, 2, 2, native.RM_SEQ_TO_HEAD)

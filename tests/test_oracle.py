@@ -361,6 +361,120 @@ def test_ulysses_layout_is_a_bijection():
     assert np.array_equal(oracle.ulysses_head_to_seq(dst), src)
 
 
+def _literal_all_to_all(shards, U, R, H):
+    """The Ulysses exchange done message by message ("Sequence Parallelism II:
+    DeepSpeed Ulysses and All-to-All Attention": before it a device has all
+    heads of some tokens, after it all tokens of some heads). shards[(r, u)]
+    is device (r, u)'s [B, s, H, D] slice; inside ring group r, device u sends
+    device u2 the heads [u2*H/U, (u2+1)*H/U) of its tokens, and u2 stacks what
+    it receives in sender order. Returns {(r, u2): [B, H/U, U*s, D]}."""
+    hU = H // U
+    inbox = {(r, u2): {} for r in range(R) for u2 in range(U)}
+    for (r, u), x in shards.items():
+        for u2 in range(U):
+            inbox[(r, u2)][u] = x[:, :, u2 * hU:(u2 + 1) * hU]      # message u -> u2
+    out = {}
+    for key, msgs in inbox.items():
+        tokens = np.concatenate([msgs[u] for u in range(U)], axis=1)  # [B, U*s, hU, D]
+        out[key] = np.ascontiguousarray(tokens.transpose(0, 2, 1, 3))
+    return out
+
+
+@pytest.mark.parametrize("U,R", [(2, 2), (4, 2), (2, 3), (1, 4), (4, 1)])
+def test_ulysses_map_equals_a_literal_all_to_all(U, R):
+    # U x R devices as separate arrays: device (r, u) starts with shard
+    # n = r*U + u (its s tokens, all heads). After a literal all-to-all inside
+    # each ring group it must hold exactly the slab [heads of u, tokens of
+    # ring rank r] of the oracle's head-sharded tensor; the way back restores
+    # every shard.
+    B, H, D = 2, 8, 3
+    s = 5
+    S = U * R * s
+    x = np.arange(B * S * H * D).reshape(B, S, H, D)
+    shards = {(r, u): x[:, (r * U + u) * s:(r * U + u + 1) * s] for r in range(R)
+              for u in range(U)}
+    held = _literal_all_to_all(shards, U, R, H)
+    full = oracle.ulysses_seq_to_head(x)
+    hU, L = H // U, S // R
+    for (r, u), got in held.items():
+        want = full[:, u * hU:(u + 1) * hU, r * L:(r + 1) * L]
+        assert np.array_equal(got, want), (r, u)
+    # the inverse exchange: device (r, u2) sends device u its token rows u*s..
+    back = {}
+    for r in range(R):
+        for u in range(U):
+            parts = [held[(r, u2)][:, :, u * s:(u + 1) * s] for u2 in range(U)]  # [B, hU, s, D]
+            back[(r, u)] = np.concatenate(parts, axis=1).transpose(0, 2, 1, 3)   # [B, s, H, D]
+    seq = oracle.ulysses_head_to_seq(full)
+    for (r, u), got in back.items():
+        n = r * U + u
+        assert np.array_equal(got, shards[(r, u)])
+        assert np.array_equal(got, seq[:, n * s:(n + 1) * s])
+
+
+def test_ulysses_literal_exchange_detects_a_planted_swap():
+    # the literal exchange is sensitive enough: swapping two heads in the
+    # oracle's map (a plausible indexing mistake) breaks the comparison
+    B, H, D, U, R, s = 1, 4, 2, 2, 2, 3
+    S = U * R * s
+    x = np.arange(B * S * H * D).reshape(B, S, H, D)
+    shards = {(r, u): x[:, (r * U + u) * s:(r * U + u + 1) * s] for r in range(R)
+              for u in range(U)}
+    held = _literal_all_to_all(shards, U, R, H)
+    wrong = oracle.ulysses_seq_to_head(x)[:, [1, 0, 2, 3]]
+    assert not np.array_equal(held[(0, 0)], wrong[:, 0:2, 0:S // R])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("order", [oracle.CONTIGUOUS, oracle.ZIGZAG])
+@pytest.mark.parametrize("P", [1, 2, 3])
+def test_step_backward_partials_sum_to_the_full_gradients(causal, order, P):
+    # The reverse ring: every (rank, owner) pair's share, summed over owners
+    # for dQ and over ranks for dK/dV, equals the oracle's dense gradients
+    # (which finite differences and torch autograd pin above).
+    S = 24 if P == 3 else 16
+    L, H, Hkv, D = S // P, 4, 2, 4
+    q, k, v, do = (_rand(sh, 80 + i) for i, sh in
+                   enumerate([(1, H, S, D), (1, Hkv, S, D), (1, Hkv, S, D), (1, H, S, D)]))
+    o, lse = oracle.attn_fwd(q, k, v, causal)
+    delta = (o * do).sum(axis=-1)
+    rdq, rdkv = oracle.attn_bwd(q, k, v, do, causal)
+    pos = oracle.rank_major_positions(S, P, order)
+    qr, kr, vr, dor, lr, dr = (x[:, :, pos] for x in (q, k, v, do, lse, delta))
+    dq = np.zeros_like(qr)
+    dk = np.zeros_like(kr)
+    dv = np.zeros_like(vr)
+    for rank in range(P):
+        sl = slice(rank * L, (rank + 1) * L)
+        for t in range(P):
+            owner = (rank - t) % P
+            blk = slice(owner * L, (owner + 1) * L)
+            a, b_, c = oracle.step_bwd_partial(qr[:, :, sl], kr[:, :, blk], vr[:, :, blk],
+                                               dor[:, :, sl], lr[:, :, sl], dr[:, :, sl], S, P,
+                                               order, rank, owner, causal)
+            dq[:, :, sl] += a
+            dk[:, :, blk] += b_
+            dv[:, :, blk] += c
+    inv = np.empty_like(pos)
+    inv[pos] = np.arange(S)
+    for h in range(H):
+        assert np.abs(dq[0, h][inv] - rdq[(0, h)]).max() < 1e-12
+    for g in range(Hkv):
+        assert np.abs(dk[0, g][inv] - rdkv[(0, g)][0]).max() < 1e-12
+        assert np.abs(dv[0, g][inv] - rdkv[(0, g)][1]).max() < 1e-12
+
+
+def test_step_backward_partial_of_an_invisible_block_is_zero():
+    # contiguous causal: rank 0's queries precede every key of owner 3
+    S, P, D = 32, 4, 4
+    L = S // P
+    q, k, v, do = _rand((1, 2, L, D), 90), _rand((1, 1, L, D), 91), _rand((1, 1, L, D), 92), \
+        _rand((1, 2, L, D), 93)
+    lse, delta = _rand((1, 2, L), 94), _rand((1, 2, L), 95)
+    for x in oracle.step_bwd_partial(q, k, v, do, lse, delta, S, P, oracle.CONTIGUOUS, 0, 3, True):
+        assert np.all(x == 0)
+
+
 # --- causal sliding window (axolotl-ringmaster README, Status: sliding-window
 # attention via flash's `window`): query i sees keys i-W < j <= i ---
 

@@ -52,6 +52,31 @@ def test_noalloc_backward_matches_workspace_backward_on_two_calls():
                          f"{name} (seed {seed})")
 
 
+def test_noalloc_backward_matches_the_oracle():
+    """The same entry point on its own against the fp64 oracle's gradients."""
+    import numpy as np
+    import oracle
+    from gpu_util import to_natural
+    from ring_ulysses_sequence_b200 import native
+    q, k, v, o, lse, do, (B, H, Hkv, S, D, P) = _problem(913)
+    dq = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    dk = torch.empty(k.shape, dtype=torch.float32, device="cuda")
+    dv = torch.empty(v.shape, dtype=torch.float32, device="cuda")
+    native.rm_ring_attn_bwd_noalloc(q, k, v, o, lse, do, dq, dk, dv, B, H, Hkv, S, D, P, True,
+                                    native.RM_ORDER_ZIGZAG, native.RM_DTYPE_BF16, D ** -0.5)
+    torch.cuda.synchronize()
+    assert native.rm_check_device_status() == native.RM_OK
+    qn, kn, vn, don = (to_natural(t.cpu(), P, "zigzag").float() for t in (q, k, v, do))
+    rdq, rdkv = oracle.attn_bwd(qn, kn, vn, don, True)
+    gq, gk, gv = (to_natural(t.cpu(), P, "zigzag").numpy() for t in (dq, dk, dv))
+    for h in range(H):
+        assert_close(gq[0, h], rdq[(0, h)], BF16_MAX_ABS, BF16_MEAN_ABS, f"dQ[{h}]")
+    for g in range(Hkv):
+        assert_close(gk[0, g], rdkv[(0, g)][0], BF16_MAX_ABS, BF16_MEAN_ABS, f"dK[{g}]")
+        assert_close(gv[0, g], rdkv[(0, g)][1], BF16_MAX_ABS, BF16_MEAN_ABS, f"dV[{g}]")
+    assert np.isfinite(gq).all()
+
+
 def test_noalloc_backward_rejects_problems_above_its_scratch():
     from ring_ulysses_sequence_b200 import native
     fake = 1 << 20  # aligned address, never touched: the size check comes first
