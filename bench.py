@@ -683,10 +683,21 @@ def bench_backward(args, dev, stream):
     torch.cuda.synchronize()
     steps = max(2, min(args.steps, 10))
     ms = time_on_stream(step, steps, stream) / steps
+    # the fused kernel (dQ by reductions), for comparison
+    before = rm.native.rm_get_bwd_deterministic()
+    rm.native.rm_set_bwd_deterministic(0)
+    try:
+        with torch.cuda.stream(stream):
+            step()
+        torch.cuda.synchronize()
+        ms_fused = time_on_stream(step, steps, stream) / steps
+    finally:
+        rm.native.rm_set_bwd_deterministic(before)
     if rm.native.rm_check_device_status(stream) != 0:
         raise RuntimeError("device watchdog fired during the backward benchmark")
     return {"workload": w.name, "ms_per_step": ms, "tflops": w.bwd_flops() / ms / 1e9,
-            "flops_per_step": w.bwd_flops()}
+            "flops_per_step": w.bwd_flops(), "ms_fused": ms_fused,
+            "tflops_fused": w.bwd_flops() / ms_fused / 1e9}
 
 
 def build_line(out, w, args, world, peaks, peak_src):
@@ -822,6 +833,9 @@ def build_line(out, w, args, world, peaks, peak_src):
         else:
             extra["ring_attn_bwd"] = {
                 "workload": b["workload"], "ms": b["ms_per_step"], "TFLOPS": b["tflops"],
+                "kernels": "two kernels, every element written once (rm_set_bwd_deterministic(1), "
+                           "the default)",
+                "ms_fused": b.get("ms_fused"), "TFLOPS_fused": b.get("tflops_fused"),
                 "roofline": {"bound": "tensor", "achieved": b["tflops"],
                              "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                              "frac": b["tflops"] / peaks["bf16_tflops_sustained"],

@@ -30,6 +30,20 @@
  *     runs out makes the kernel stop early, write nothing further and set a
  *     device status word that rm_check_device_status() reports as
  *     RM_ERR_TIMEOUT. Outputs of such a call are undefined.
+ *   - Launches in flight. The attention kernels (forward, backward and their
+ *     step variants) are persistent: their blocks take work items from a
+ *     counter in device memory. The library keeps 256 such counters per
+ *     device and gives each launch the next one in turn, re-armed on the
+ *     launch's stream just before it. So at most 256 of these launches may be
+ *     in flight at once on a device (on any streams). A CUDA graph that
+ *     captured a launch keeps that launch's counter: replays of one graph must
+ *     not overlap each other, and a replay must not overlap the 256th eager
+ *     launch after the capture. A launch whose counter is re-armed by another
+ *     one while it runs notices it, stops taking work (its outputs are
+ *     undefined) and sets the status word, which rm_check_device_status()
+ *     reports as RM_ERR_SLOT_REUSE; the other launch is not disturbed.
+ *     (Overlapping replays of one graph re-arm with the same value and cannot
+ *     be told apart.)
  */
 #ifndef RM_H
 #define RM_H
@@ -53,7 +67,8 @@ typedef enum rm_status {
     RM_ERR_INVALID_ARG = 1,  /* null pointer, bad size, bad enum, misalignment */
     RM_ERR_UNSUPPORTED = 2,  /* valid request outside the shapes/dtypes built */
     RM_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
-    RM_ERR_TIMEOUT = 4       /* a bounded in-kernel wait ran out */
+    RM_ERR_TIMEOUT = 4,      /* a bounded in-kernel wait ran out */
+    RM_ERR_SLOT_REUSE = 5    /* more launches in flight than work-counter slots */
 } rm_status;
 
 /* Token order of the ring ("context parallelism", Last Dictionary: causal
@@ -491,13 +506,29 @@ RM_API rm_status rm_seq_reorder(const void* src, void* dst, int B, int H, int S,
                          cudaStream_t stream);
 
 /* Synchronises `stream`, then reads and clears the device status word of the
- * current device. Returns RM_ERR_TIMEOUT if a bounded wait ran out since the
- * last check, RM_ERR_CUDA if the synchronisation failed, else RM_OK. */
+ * current device. Returns RM_ERR_SLOT_REUSE if a launch found its work counter
+ * re-armed by another launch since the last check, else RM_ERR_TIMEOUT if a
+ * bounded wait ran out, RM_ERR_CUDA if the synchronisation failed, else
+ * RM_OK. */
 RM_API rm_status rm_check_device_status(cudaStream_t stream);
 
 /* Limit for every in-kernel wait, in nanoseconds (default 2e9). Applies to
  * launches made after the call; values below 1000 are raised to 1000. */
 RM_API void rm_set_watchdog_ns(uint64_t ns);
+
+/* Which kernels the backward entry points (rm_ring_attn_bwd*, including the
+ * window, varlen, no-alloc and step variants) use, process-wide, for calls
+ * made after this one. 1 (the default): two kernels (KV-stationary dK/dV,
+ * Q-stationary dQ) that write every gradient element exactly once, so the
+ * result is bitwise reproducible. 0: one fused kernel that computes S and dP
+ * once per tile pair (five tensor-core products instead of seven) and adds dQ
+ * into place with fp32 reductions at L2 (TMA reduce-add); the order of those
+ * additions varies between runs, so dQ may differ in its last bits from run
+ * to run (dK and dV do not). On B200 the reductions (64 KB per 128 x 128 tile
+ * pair) cost more than the two products they save, so the fused kernel is the
+ * slower of the two. */
+RM_API void rm_set_bwd_deterministic(int on);
+RM_API int rm_get_bwd_deterministic(void);
 
 /* Launches one kernel that waits on a barrier nothing will complete, bounded
  * by timeout_ns, so that callers can see the watchdog path end in

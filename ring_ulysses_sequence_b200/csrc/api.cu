@@ -14,14 +14,18 @@ __device__ unsigned g_status_word;
 __device__ int g_work_counters[kWorkSlots];
 static std::atomic<uint32_t> g_work_seq{0};
 
-cudaError_t next_work_counter(const LaunchCtx& ctx, int** counter) {
-    int* c = ctx.work_counters + (g_work_seq.fetch_add(1) % kWorkSlots);
-    *counter = c;
-    return cudaMemsetAsync(c, 0, sizeof(int), ctx.stream);
+cudaError_t next_work_counter(const LaunchCtx& ctx, int n_items, WorkCounter* counter) {
+    const uint32_t seq = g_work_seq.fetch_add(1);
+    const int gen = static_cast<int>((seq / kWorkSlots) % 255u) + 1;  // 1..255, in every byte
+    counter->ptr = ctx.work_counters + (seq % kWorkSlots);
+    counter->base = gen * 0x01010101;
+    counter->n_items = n_items;
+    return cudaMemsetAsync(counter->ptr, gen, sizeof(int), ctx.stream);
 }
 
 static thread_local int t_last_cuda_error = 0;
 static std::atomic<uint64_t> g_watchdog_ns{2000000000ull};
+static std::atomic<int> g_bwd_deterministic{1};
 
 static rm_status cuda_fail(cudaError_t e) {
     t_last_cuda_error = static_cast<int>(e);
@@ -176,6 +180,7 @@ const char* rm_status_string(rm_status s) {
         case RM_ERR_UNSUPPORTED: return "unsupported shape or dtype";
         case RM_ERR_CUDA: return "CUDA error";
         case RM_ERR_TIMEOUT: return "in-kernel wait timed out";
+        case RM_ERR_SLOT_REUSE: return "more launches in flight than work-counter slots";
     }
     return "unknown status";
 }
@@ -183,6 +188,10 @@ const char* rm_status_string(rm_status s) {
 int rm_last_cuda_error(void) { return t_last_cuda_error; }
 
 void rm_set_watchdog_ns(uint64_t ns) { g_watchdog_ns.store(ns < 1000 ? 1000 : ns); }
+
+void rm_set_bwd_deterministic(int on) { g_bwd_deterministic.store(on ? 1 : 0); }
+
+int rm_get_bwd_deterministic(void) { return g_bwd_deterministic.load(); }
 
 rm_status rm_check_device_status(cudaStream_t stream) {
     LaunchCtx ctx;
@@ -197,7 +206,7 @@ rm_status rm_check_device_status(cudaStream_t stream) {
         const unsigned zero = 0;
         e = cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero));
         if (e != cudaSuccess) return cuda_fail(e);
-        return RM_ERR_TIMEOUT;
+        return (word & kErrSlotReuse) ? RM_ERR_SLOT_REUSE : RM_ERR_TIMEOUT;
     }
     return RM_OK;
 }
@@ -356,6 +365,7 @@ static rm_status bwd_impl(const void* q, const void* k, const void* v, const voi
     if ((st = get_ctx(stream, &ctx)) != RM_OK) return st;
     AttnShape sh{B, H, Hkv, S, D, P, causal ? 1 : 0, order == RM_ORDER_ZIGZAG ? 1 : 0, scale,
                  window, bounds};
+    sh.deterministic = g_bwd_deterministic.load();
     cudaError_t e = launch_bwd(sh, q, k, v, o, lse, dout, dq, dk, dv,
                                static_cast<float*>(workspace), ctx);
     return e == cudaSuccess ? RM_OK : cuda_fail(e);
@@ -382,6 +392,7 @@ rm_status rm_ring_attn_bwd_noalloc(const void* q, const void* k, const void* v, 
     float* scratch = nullptr;
     if ((st = noalloc_scratch(&scratch)) != RM_OK) return st;
     AttnShape sh{B, H, Hkv, S, D, P, causal ? 1 : 0, order == RM_ORDER_ZIGZAG ? 1 : 0, scale};
+    sh.deterministic = g_bwd_deterministic.load();
     // Delta is rewritten in full by the backward's first kernel, so the
     // previous call's contents need no clearing.
     cudaError_t e = launch_bwd(sh, q, k, v, o, lse, dout, dq, dk, dv, scratch, ctx);
@@ -422,6 +433,7 @@ rm_status rm_ring_attn_bwd_step(const void* q_local, const void* k_block, const 
     if ((st = get_ctx(stream, &ctx)) != RM_OK) return st;
     AttnShape sh{B, H, Hkv, S, D, P, causal ? 1 : 0, order == RM_ORDER_ZIGZAG ? 1 : 0, scale, 0,
                  nullptr, 2, rank, owner, 0};
+    sh.deterministic = g_bwd_deterministic.load();
     cudaError_t e = launch_bwd(sh, q_local, k_block, v_block, nullptr, lse_local, dout_local,
                                dq_local, dk_block, dv_block, const_cast<float*>(delta_local), ctx);
     return e == cudaSuccess ? RM_OK : cuda_fail(e);

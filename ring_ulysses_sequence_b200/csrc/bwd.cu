@@ -81,13 +81,14 @@ __device__ __forceinline__ uint32_t packed_col(int k) { return k < 4 ? 8 * k : 6
 
 struct BwdArgs {
     CUtensorMap tm_q, tm_k, tm_v, tm_do;
+    CUtensorMap tm_dq;  // fused kernel: fp32 dQ in 128-row x 32-column boxes (TMA reduce-add)
     const float* lse;
     const float* delta;
     float* dq;
     float* dk;
     float* dv;
     unsigned* status;
-    int* work;       // this launch's work-item counter
+    WorkCounter work;  // this launch's work-item counter
     unsigned long long timeout_ns;
     int B, H, Hkv, S, P, causal, G, n_items;
     MaskSpec mk;     // which keys each query sees
@@ -543,6 +544,474 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
     }
 }
 
+// -------------------------------------------------------------------- fused
+
+// One kernel for dK, dV and dQ: five products per tile pair instead of the
+// seven of the two kernels (S and dP are computed once). It is KV-stationary
+// like ring_bwd_dkdv_kernel; in addition the compute warps write dS^T as bf16
+// to shared memory, where it is the A operand of both dK += dS^T Q (read
+// K-major) and dQ_tile = dS K (the same bytes read MN-major, i.e. transposed).
+// dQ_tile lands in the TMEM columns of dP^T, which the compute warps have read
+// by then. They read it out, scale it, and write it 64 columns at a time to a
+// 32 KB staging tile, which a reducer thread adds into global dQ with TMA
+// reduce-add (fp32 additions at L2, whole 128-byte lines; per-thread vector
+// reductions instead issue 4096 separate 16-byte requests per tile pair, which
+// the SM's path to L2 cannot sustain). The order of those additions across
+// CTAs depends on timing, so dQ varies in its last bits from run to run; dK
+// and dV are written once per element. The two-kernel path is the
+// deterministic option.
+//
+// Roles: warps 0-7 compute (two warpgroups, 64 query columns each), warp 8
+// lane 0 issues UMMA, warp 9 lane 0 loads by TMA, warp 9 lane 1 issues the dQ
+// reductions. TMEM: S^T [0,128) (bf16 P^T over it), dP^T then dQ_tile
+// [128,256), dV at 256, dK at 384. Shared memory: K, V resident; two stages of
+// Q + dO; the dQ staging tile (128 rows x 64 fp32, two 32-column boxes with
+// the 128-byte swizzle). dS^T (128 x 128 bf16, laid out like a TMA tile) goes
+// over the stage's dO once dV has read it when D = 128 (dO is then exactly
+// its size); with D = 64 it has a buffer of its own. LSE and Delta come
+// straight from global memory (every thread of a warpgroup reads the same 64
+// values).
+constexpr int kDsBox = kT * 128;  // one 64-column box of the dS^T tile; one 32-column fp32 box
+
+template <int D>
+struct FCfg {
+    static constexpr bool kDsInStage = D == 128;      // dS^T over the stage's dO
+    static constexpr int kTile = kT * D * 2;
+    static constexpr int kStage = 2 * kTile;          // Q + dO
+    static constexpr int kStOff = 2 * kTile;
+    static constexpr int kStgOff = kStOff + kStages * kStage;
+    static constexpr int kDsOff = kStgOff + kT * 64 * 4;  // own dS^T buffer (D = 64)
+    static constexpr int kBarOff = kDsOff + (kDsInStage ? 0 : kT * kT * 2);
+    static constexpr int kSmem = kBarOff + 256 + 1024;
+};
+static_assert(FCfg<128>::kSmem <= 232448, "shared memory of the fused backward");
+static_assert(FCfg<64>::kSmem <= 232448, "shared memory of the fused backward");
+
+struct FBars {
+    ItemRing items;
+    uint64_t res_full, res_empty, drain, acc_full;
+    uint64_t st_full[kStages], st_empty[kStages];
+    uint64_t s_full, dp_full;  // S^T, dP^T in TMEM
+    uint64_t p_half;           // P^T written (256 arrivals)
+    uint64_t dv_done;          // dV has read the stage's dO (dS^T may overwrite it)
+    uint64_t ds_full;          // dS^T in shared memory and dP^T read out (256)
+    uint64_t dq_full;          // dK and dQ_tile done: dQ_tile in TMEM, dS^T and the stage free
+    uint64_t dq_empty;         // dQ_tile read out of TMEM (256)
+    uint64_t stg_full;         // a 64-column round of dQ_tile staged (256)
+    uint64_t stg_free;         // the reducer's TMA has read the staging tile (1)
+    int stg_row;               // the round's first dQ row (-1: no more), and which round
+    int stg_round;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+static_assert(sizeof(FBars) <= 256, "barrier block");
+
+template <int D>
+__device__ __forceinline__ void issue_dk_product(uint32_t tmem_acc, uint32_t ds_smem, uint32_t q_smem,
+                                                 bool accumulate) {
+    // dK[128 keys x D] += dS^T[128 keys x 128 queries] (K-major) * Q[128 queries x D] (MN-major)
+    constexpr uint32_t idesc = umma_idesc_bf16(kT, D, 0, 1);
+#pragma unroll
+    for (int k = 0; k < kT / 16; ++k)
+        umma_ss(tmem_acc, umma_desc_sw128(ds_smem + (k >> 2) * kDsBox + (k & 3) * 32, 16, 1024),
+                umma_desc_sw128(q_smem + k * 2048, BCfg<D>::kBox, 1024), idesc,
+                (accumulate || k > 0) ? 1u : 0u);
+}
+
+template <int D>
+__device__ __forceinline__ void issue_dq_product(uint32_t tmem_acc, uint32_t ds_smem, uint32_t k_smem) {
+    // dQ_tile[128 queries x D] = dS[128 queries x 128 keys] (MN-major: the dS^T
+    // bytes) * K[128 keys x D] (MN-major)
+    constexpr uint32_t idesc = umma_idesc_bf16(kT, D, 1, 1);
+#pragma unroll
+    for (int k = 0; k < kT / 16; ++k)
+        umma_ss(tmem_acc, umma_desc_sw128(ds_smem + k * 2048, kDsBox, 1024),
+                umma_desc_sw128(k_smem + k * 2048, BCfg<D>::kBox, 1024), idesc, k > 0 ? 1u : 0u);
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) ring_bwd_fused_kernel(const __grid_constant__ BwdArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    FBars& bars = *reinterpret_cast<FBars*>(smem + FCfg<D>::kBarOff);
+    const uint32_t k_smem = smem_u32(smem);
+    const uint32_t v_smem = k_smem + FCfg<D>::kTile;
+    const uint32_t st_smem = k_smem + FCfg<D>::kStOff;   // stage s: Q, dO
+    const uint32_t stg_smem = k_smem + FCfg<D>::kStgOff;  // dQ staging (two 32-column fp32 boxes)
+    // dS^T of a tile in stage st: over its dO (D = 128) or in the own buffer (D = 64)
+    auto ds_of = [&](int st) -> uint32_t {
+        return FCfg<D>::kDsInStage ? st_smem + st * FCfg<D>::kStage + FCfg<D>::kTile
+                                   : k_smem + FCfg<D>::kDsOff;
+    };
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        bars.abort_flag = 0;
+        item_ring_init(bars.items, kItemReaders);
+        mbar_init(smem_u32(&bars.res_full), 1);
+        mbar_init(smem_u32(&bars.res_empty), 1);
+        mbar_init(smem_u32(&bars.drain), 1);
+        mbar_init(smem_u32(&bars.acc_full), 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(smem_u32(&bars.st_full[s]), 1);
+            mbar_init(smem_u32(&bars.st_empty[s]), 1);
+        }
+        mbar_init(smem_u32(&bars.s_full), 1);
+        mbar_init(smem_u32(&bars.dp_full), 1);
+        mbar_init(smem_u32(&bars.p_half), 256);
+        mbar_init(smem_u32(&bars.dv_done), 1);
+        mbar_init(smem_u32(&bars.ds_full), 256);
+        mbar_init(smem_u32(&bars.dq_full), 1);
+        mbar_init(smem_u32(&bars.dq_empty), 256);
+        mbar_init(smem_u32(&bars.stg_full), 256);
+        mbar_init(smem_u32(&bars.stg_free), 1);
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&bars.tmem_base), 512);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars.tmem_base;
+    const Watchdog wd{a.status, &bars.abort_flag, a.timeout_ns};
+
+    if (warp == kLoadWarp) {
+        if (lane == 0) {
+            // ------------------------------------------------------ producer
+            prefetch_tmap(&a.tm_q);
+            prefetch_tmap(&a.tm_k);
+            prefetch_tmap(&a.tm_v);
+            prefetch_tmap(&a.tm_do);
+            uint32_t items = 0, fills = 0;
+            bool ok = true;
+            for (uint32_t k = 0; ok; ++k) {
+                int w;
+                ok = item_claim(bars.items, a.work, k, w, wd);
+                if (!ok || w >= a.n_items) break;
+                const KvItem it = decode_kv_item(a, w);
+                QIter qi(a, it);
+                int h, qslot, cls;
+                bool more = qi.next(a, h, qslot, cls);
+                if (!more) continue;  // one step: no query of the rank sees this tile
+                if (items > 0) ok = mbar_wait(smem_u32(&bars.res_empty), (items - 1) & 1, wd);
+                if (!ok) break;
+                ++items;
+                const int krow = (it.b * a.Hkv + it.g) * a.kv_len + it.kslot;
+                mbar_arrive_expect_tx(smem_u32(&bars.res_full), 2 * FCfg<D>::kTile);
+                for (int bx = 0; bx < BCfg<D>::kBoxes; ++bx) {
+                    tma_load_2d(k_smem + bx * BCfg<D>::kBox, &a.tm_k, bx * 64, krow, smem_u32(&bars.res_full));
+                    tma_load_2d(v_smem + bx * BCfg<D>::kBox, &a.tm_v, bx * 64, krow, smem_u32(&bars.res_full));
+                }
+                for (; ok && more; more = qi.next(a, h, qslot, cls)) {
+                    const int st = fills % kStages;
+                    const uint32_t use = fills / kStages;
+                    if (use > 0) ok = mbar_wait(smem_u32(&bars.st_empty[st]), (use - 1) & 1, wd);
+                    if (!ok) break;
+                    const uint32_t base = st_smem + st * FCfg<D>::kStage;
+                    const int qrow = (it.b * a.H + h) * a.q_len + qslot;
+                    const uint32_t bar = smem_u32(&bars.st_full[st]);
+                    mbar_arrive_expect_tx(bar, FCfg<D>::kStage);
+                    for (int bx = 0; bx < BCfg<D>::kBoxes; ++bx) {
+                        tma_load_2d(base + bx * BCfg<D>::kBox, &a.tm_q, bx * 64, qrow, bar);
+                        tma_load_2d(base + FCfg<D>::kTile + bx * BCfg<D>::kBox, &a.tm_do, bx * 64, qrow, bar);
+                    }
+                    ++fills;
+                }
+            }
+            if (!ok) {
+                volatile int no_abort = 0;
+                const Watchdog w2{a.status, &no_abort, a.timeout_ns};
+                for (uint32_t i = fills > kStages ? fills - kStages : 0; i < fills; ++i)
+                    (void)mbar_wait(smem_u32(&bars.st_full[i % kStages]), (i / kStages) & 1, w2);
+                if (items > 0) (void)mbar_wait(smem_u32(&bars.res_full), (items - 1) & 1, w2);
+            }
+        } else if (lane == 1) {
+            // ------------------------------------------------------ dQ reducer
+            // Adds each staged 64-column round into global dQ (box 0 -> columns
+            // 32 r, box 1 -> D/2 + 32 r for round r), and frees the staging tile
+            // once the TMA has read it. Single-thread role: no warp-collective
+            // operation here.
+            prefetch_tmap(&a.tm_dq);
+            for (uint32_t n = 0;; ++n) {
+                if (!mbar_wait(smem_u32(&bars.stg_full), n & 1, wd)) break;
+                const int row = *reinterpret_cast<volatile int*>(&bars.stg_row);
+                const int round = *reinterpret_cast<volatile int*>(&bars.stg_round);
+                if (row < 0) break;
+                tma_reduce_add_2d(&a.tm_dq, 32 * round, row, stg_smem);
+                tma_reduce_add_2d(&a.tm_dq, D / 2 + 32 * round, row, stg_smem + kDsBox);
+                bulk_commit_group();
+                bulk_wait_read_all();
+                mbar_arrive(smem_u32(&bars.stg_free));
+            }
+            bulk_wait_all();  // every reduction issued has landed before the CTA exits
+        }
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            // ------------------------------------------------------ MMA issuer
+            const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 384;
+            uint32_t items = 0, uses = 0, p_cnt = 0, dq_cnt = 0;
+            bool ok = true;
+            for (uint32_t k = 0; ok; ++k) {
+                int w;
+                ok = item_read(bars.items, k, w, false, wd);
+                if (!ok || w >= a.n_items) break;
+                const KvItem it = decode_kv_item(a, w);
+                QIter qi(a, it);
+                int qh, qs, qc;
+                if (!qi.next(a, qh, qs, qc)) continue;  // query tile 0 (one step may have none)
+                ok = mbar_wait(smem_u32(&bars.res_full), items & 1, wd);
+                if (!ok) break;
+                ++items;
+                tc_fence_after();
+                auto stage = [&](int& st) -> bool {
+                    st = uses % kStages;
+                    const bool r = mbar_wait(smem_u32(&bars.st_full[st]), (uses / kStages) & 1, wd);
+                    ++uses;
+                    tc_fence_after();
+                    return r;
+                };
+                int st = 0;
+                ok = stage(st);
+                if (ok) {
+                    const uint32_t q_addr = st_smem + st * FCfg<D>::kStage;
+                    issue_tile_product<D>(tS, k_smem, q_addr);  // S^T = K Q^T
+                    umma_commit(smem_u32(&bars.s_full));
+                    // dP^T goes where the previous tile's dQ was: it must be read out
+                    if (dq_cnt > 0) ok = mbar_wait(smem_u32(&bars.dq_empty), (dq_cnt - 1) & 1, wd);
+                    if (ok) {
+                        tc_fence_after();
+                        issue_tile_product<D>(tdP, v_smem, q_addr + FCfg<D>::kTile);  // dP^T = V dO^T
+                        umma_commit(smem_u32(&bars.dp_full));
+                    }
+                }
+                for (int j = 0; ok; ++j) {
+                    const uint32_t q_addr = st_smem + st * FCfg<D>::kStage;
+                    const uint32_t do_addr = q_addr + FCfg<D>::kTile;
+                    ok = mbar_wait(smem_u32(&bars.p_half), p_cnt & 1, wd);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_acc_product<D>(tdV, tS, do_addr, j > 0);  // dV += P^T dO
+                    umma_commit(smem_u32(&bars.dv_done));          // dO read: dS^T may go there
+                    const bool have_next = qi.next(a, qh, qs, qc);
+                    int st_next = st;
+                    if (have_next) {  // S^T of the next tile overwrites P^T after dV read it
+                        ok = stage(st_next);
+                        if (!ok) break;
+                        issue_tile_product<D>(tS, k_smem, st_smem + st_next * FCfg<D>::kStage);
+                        umma_commit(smem_u32(&bars.s_full));
+                    }
+                    ok = mbar_wait(smem_u32(&bars.ds_full), (p_cnt++) & 1, wd);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_dk_product<D>(tdK, ds_of(st), q_addr, j > 0);  // dK += dS^T Q
+                    issue_dq_product<D>(tdP, ds_of(st), k_smem);          // dQ_tile = dS K
+                    umma_commit(smem_u32(&bars.st_empty[st]));            // Q and dS^T read
+                    umma_commit(smem_u32(&bars.dq_full));
+                    ++dq_cnt;
+                    if (!have_next) break;
+                    ok = mbar_wait(smem_u32(&bars.dq_empty), (dq_cnt - 1) & 1, wd);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_tile_product<D>(tdP, v_smem, st_smem + st_next * FCfg<D>::kStage + FCfg<D>::kTile);
+                    umma_commit(smem_u32(&bars.dp_full));
+                    st = st_next;
+                }
+                if (!ok) break;
+                umma_commit(smem_u32(&bars.acc_full));
+                umma_commit(smem_u32(&bars.res_empty));  // after dQ_tile, the last reader of K
+            }
+            umma_commit(smem_u32(&bars.drain));
+            volatile int no_abort = 0;
+            const Watchdog w2{a.status, &no_abort, a.timeout_ns};
+            (void)mbar_wait(smem_u32(&bars.drain), 0, w2);
+        }
+    } else {
+        // ---------------------------------------------------------- compute
+        const int wg = warp >> 2;               // which 64 query columns (and D/2 dQ columns)
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;      // TMEM lane: key row (S^T, dP^T), query row (dQ)
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        const uint32_t tS = tmem + lane_off + 64 * wg;
+        const uint32_t tdP = tmem + lane_off + 128 + 64 * wg;
+        constexpr int HC = D / 2;               // accumulator columns per warpgroup
+        const uint32_t tdQ = tmem + lane_off + 128 + HC * wg;
+        const uint32_t tdV = tmem + lane_off + 256 + HC * wg;
+        const uint32_t tdK = tmem + lane_off + 384 + HC * wg;
+        const uint32_t stg_row = stg_smem + wg * kDsBox + r * 128;  // this thread's staging row
+        const float sl2 = a.scale_log2;
+        uint32_t uses = 0, s_cnt = 0, items = 0, dq_cnt = 0, rounds = 0;
+        // dQ_tile of the tile before: waits for dK and dQ_tile, reads it out of
+        // TMEM (then dP^T of the next tile may go there) and stages it, scaled,
+        // 32 of this thread's columns per round, for the reducer.
+        auto drain = [&](int row) -> bool {
+            if (!mbar_wait(smem_u32(&bars.dq_full), dq_cnt & 1, wd)) return false;
+            ++dq_cnt;
+            tc_fence_after();
+#pragma unroll
+            for (int rd = 0; rd < HC / 32; ++rd) {
+                uint32_t v[32];
+                tmem_ld32(tdQ + 32 * rd, v);
+                if (rd == HC / 32 - 1) {  // all of dQ_tile read out: dP^T may overwrite it
+                    tc_fence_before();
+                    mbar_arrive(smem_u32(&bars.dq_empty));
+                }
+                // the previous round's TMA has read the staging tile
+                if (rounds > 0 && !mbar_wait(smem_u32(&bars.stg_free), (rounds - 1) & 1, wd)) return false;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    st_shared_v4(stg_row + ((c ^ (r & 7)) << 4),
+                                 __float_as_uint(__uint_as_float(v[4 * c]) * a.scale),
+                                 __float_as_uint(__uint_as_float(v[4 * c + 1]) * a.scale),
+                                 __float_as_uint(__uint_as_float(v[4 * c + 2]) * a.scale),
+                                 __float_as_uint(__uint_as_float(v[4 * c + 3]) * a.scale));
+                fence_proxy_async_smem();
+                if (threadIdx.x == 0) {
+                    bars.stg_row = row;
+                    bars.stg_round = rd;
+                }
+                mbar_arrive(smem_u32(&bars.stg_full));
+                ++rounds;
+            }
+            return true;
+        };
+        bool ok = true;
+        for (uint32_t k = 0; ok; ++k) {
+            int w;
+            ok = item_read(bars.items, k, w, true, wd);
+            if (!ok || w >= a.n_items) break;
+            const KvItem it = decode_kv_item(a, w);
+            QIter qi(a, it);
+            int h, qslot, cls, ntiles = 0, pend_row = -1;
+            while (ok && qi.next(a, h, qslot, cls)) {
+                const int st = uses % kStages;
+                ++uses;
+                // key row r sees query column c iff imin(j) <= qpos + c <= imax(j)
+                int lo = 0;
+                unsigned wq = 0;
+                if (cls == kMask) {
+                    const int2 cb = col_bounds(a.mk, it.kpos + r);
+                    lo = cb.x - qi.qpos;
+                    wq = static_cast<unsigned>(cb.y - cb.x);
+                }
+                const int qrow0 = (it.b * a.H + h) * a.q_len + qslot;
+                const float4* lse4 = reinterpret_cast<const float4*>(a.lse + qrow0 + 64 * wg);
+                const float4* del4 = reinterpret_cast<const float4*>(a.delta + qrow0 + 64 * wg);
+                ok = mbar_wait(smem_u32(&bars.s_full), s_cnt & 1, wd);
+                if (!ok) break;
+                tc_fence_after();
+                // P^T from S^T and LSE, bf16 over the S^T columns already read
+                const uint64_t sl2x2 = pk2(sl2, sl2);
+                const uint64_t nlog2e = pk2(-kLog2e, -kLog2e);
+                uint64_t pp[32];  // P of this thread's 64 query columns, in pairs
+#pragma unroll
+                for (int qq = 0; qq < 2; ++qq) {
+                    uint32_t sv[32];
+                    tmem_ld32(tS + 32 * qq, sv);
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        const float4 L = __ldg(lse4 + 8 * qq + c4);
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const int c = 4 * c4 + 2 * hh;
+                            const uint64_t lse2 = mul2(hh ? pk2(L.z, L.w) : pk2(L.x, L.y), nlog2e);
+                            float x0, x1;
+                            upk2(fma2(pk2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, lse2), x0, x1);
+                            float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                            if (cls == kMask) {
+                                const int q0 = 64 * wg + 32 * qq + c;
+                                if (static_cast<unsigned>(q0 - lo) > wq) p0 = 0.f;
+                                if (static_cast<unsigned>(q0 + 1 - lo) > wq) p1 = 0.f;
+                            }
+                            pp[16 * qq + (c >> 1)] = pk2(p0, p1);
+                            pk[c >> 1] = pack_bf16x2(p0, p1);
+                        }
+                    }
+                    tmem_st16(tS + 16 * qq, pk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(smem_u32(&bars.p_half));
+                // the previous tile's dQ_tile, while this tile's dV runs
+                if (pend_row >= 0) {
+                    ok = drain(pend_row);
+                    if (!ok) break;
+                }
+                ok = mbar_wait(smem_u32(&bars.dp_full), (s_cnt++) & 1, wd);
+                if (!ok) break;
+                tc_fence_after();
+                if constexpr (FCfg<D>::kDsInStage) {  // dS^T goes over dO: dV must have read it
+                    ok = mbar_wait(smem_u32(&bars.dv_done), (s_cnt - 1) & 1, wd);
+                    if (!ok) break;
+                }
+                // dS^T = P^T (dP^T - Delta), bf16, to shared memory (the swizzled
+                // layout of a TMA tile: 16-byte chunk c of row r at c ^ (r % 8))
+                const uint32_t ds_row = ds_of(st) + wg * kDsBox + r * 128;
+#pragma unroll
+                for (int qq = 0; qq < 2; ++qq) {
+                    uint32_t dpv[32];
+                    tmem_ld32(tdP + 32 * qq, dpv);
+                    uint32_t dsk[16];
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        const float4 Dl = __ldg(del4 + 8 * qq + c4);
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const int c = 4 * c4 + 2 * hh;
+                            const uint64_t dd = mul2(pp[16 * qq + (c >> 1)],
+                                                     sub2(pk2(__uint_as_float(dpv[c]), __uint_as_float(dpv[c + 1])),
+                                                          hh ? pk2(Dl.z, Dl.w) : pk2(Dl.x, Dl.y)));
+                            float d0, d1;
+                            upk2(dd, d0, d1);
+                            dsk[c >> 1] = pack_bf16x2(d0, d1);
+                        }
+                    }
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc)
+                        st_shared_v4(ds_row + (((4 * qq + cc) ^ (r & 7)) << 4), dsk[4 * cc],
+                                     dsk[4 * cc + 1], dsk[4 * cc + 2], dsk[4 * cc + 3]);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(smem_u32(&bars.ds_full));
+                pend_row = qrow0;
+                ++ntiles;
+            }
+            if (!ok) break;
+            if (ntiles == 0) continue;  // one step: the tile meets none of the rank's queries
+            ok = drain(pend_row);
+            if (!ok) break;
+            ok = mbar_wait(smem_u32(&bars.acc_full), items & 1, wd);
+            if (!ok) break;
+            ++items;
+            tc_fence_after();
+            const int64_t krow = (static_cast<int64_t>(it.b) * a.Hkv + it.g) * a.kv_len + it.kslot + r;
+            store_cols<HC>(tdV, a.dv + krow * D + HC * wg, 1.0f, a.step);
+            store_cols<HC>(tdK, a.dk + krow * D + HC * wg, a.scale, a.step);
+        }
+        if (ok) {  // no more work: the reducer stops at this sentinel
+            if (rounds > 0) ok = mbar_wait(smem_u32(&bars.stg_free), (rounds - 1) & 1, wd);
+            if (ok && threadIdx.x == 0) bars.stg_row = -1;
+            if (ok) mbar_arrive(smem_u32(&bars.stg_full));
+        }
+    }
+
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
 // -------------------------------------------------------------------- dQ
 
 struct QItem {
@@ -946,7 +1415,7 @@ cudaError_t launch_bwd_d(const AttnShape& sh, const BwdArgs& base, const void* o
 
     BwdArgs a = base;
     a.n_items = sh.B * sh.Hkv * (a.kv_len / kT);
-    if ((e = next_work_counter(ctx, &a.work)) != cudaSuccess) return e;
+    if ((e = next_work_counter(ctx, a.n_items, &a.work)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(ring_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   BCfg<D>::kSmemKV)) != cudaSuccess)
         return e;
@@ -954,11 +1423,33 @@ cudaError_t launch_bwd_d(const AttnShape& sh, const BwdArgs& base, const void* o
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     a.n_items = sh.B * sh.H * (a.q_len / kT);
-    if ((e = next_work_counter(ctx, &a.work)) != cudaSuccess) return e;
+    if ((e = next_work_counter(ctx, a.n_items, &a.work)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(ring_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   BCfg<D>::kSmemQ)) != cudaSuccess)
         return e;
     ring_bwd_dq_kernel<D><<<std::min(a.n_items, ctx.num_sms), kThreads, BCfg<D>::kSmemQ, ctx.stream>>>(a);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_bwd_fused(const AttnShape& sh, const BwdArgs& base, const void* o,
+                             const void* dout, float* delta, float* dq, const LaunchCtx& ctx) {
+    cudaError_t e;
+    if (!base.step) {
+        const int64_t rows = static_cast<int64_t>(sh.B) * sh.H * sh.S;
+        if ((e = launch_delta<D, __nv_bfloat16>(o, dout, delta, rows, ctx)) != cudaSuccess) return e;
+        // dQ is a sum of reductions: it starts at zero (one step adds to the caller's)
+        if ((e = cudaMemsetAsync(dq, 0, static_cast<size_t>(rows) * D * sizeof(float), ctx.stream)) !=
+            cudaSuccess)
+            return e;
+    }
+    BwdArgs a = base;
+    a.n_items = sh.B * sh.Hkv * (a.kv_len / kT);
+    if ((e = next_work_counter(ctx, a.n_items, &a.work)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(ring_bwd_fused_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  FCfg<D>::kSmem)) != cudaSuccess)
+        return e;
+    ring_bwd_fused_kernel<D><<<std::min(a.n_items, ctx.num_sms), kThreads, FCfg<D>::kSmem, ctx.stream>>>(a);
     return cudaGetLastError();
 }
 
@@ -1000,6 +1491,11 @@ cudaError_t launch_bwd(const AttnShape& sh, const void* q, const void* k, const 
     a.owner = step ? sh.owner : 0;
     a.q_len = len;
     a.kv_len = len;
+    if (!sh.deterministic) {
+        if ((e = make_tmap_f32_rows(&a.tm_dq, dq, qrows, sh.D, kT, 32)) != cudaSuccess) return e;
+        return sh.D == 64 ? launch_bwd_fused<64>(sh, a, o, dout, delta, dq, ctx)
+                          : launch_bwd_fused<128>(sh, a, o, dout, delta, dq, ctx);
+    }
     return sh.D == 64 ? launch_bwd_d<64>(sh, a, o, dout, delta, ctx)
                       : launch_bwd_d<128>(sh, a, o, dout, delta, ctx);
 }

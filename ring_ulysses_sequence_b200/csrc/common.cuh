@@ -93,7 +93,7 @@ __host__ __device__ __forceinline__ int ceil_div128(int x) { return -((-x) >> 7)
 // Watchdog: every spin-wait is bounded in time.
 // ---------------------------------------------------------------------------
 
-enum : unsigned { kErrTimeout = 1u };
+enum : unsigned { kErrTimeout = 1u, kErrSlotReuse = 2u };
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
@@ -187,13 +187,46 @@ __device__ __forceinline__ void item_ring_init(ItemRing& r, int readers) {
     }
 }
 
-// Claims the k-th item of this CTA (one thread).
-__device__ __forceinline__ bool item_claim(ItemRing& r, int* counter, uint32_t k, int& w,
+// A launch's work-item counter: one of the library's counter slots, set to
+// `base` on the launch's stream just before the launch. base carries the
+// launch's generation in every byte (g * 0x01010101, g = 1..255), and two
+// launches that use one slot one after the other have different generations.
+// Every claim before the last returns an index below n_items and each CTA
+// makes one claim past it, so a value outside [base, base + n_items + grid]
+// means another launch has re-armed the slot while this one still runs.
+struct WorkCounter {
+    int* ptr;
+    int base;
+    int n_items;
+};
+
+// Claims the k-th item of this CTA (one thread). The compare-and-swap only
+// advances a counter that still belongs to this launch: a launch that finds
+// its slot re-armed raises kErrSlotReuse and takes no item from the other
+// launch (it publishes n_items, "no more work", and stops).
+__device__ __forceinline__ bool item_claim(ItemRing& r, const WorkCounter& c, uint32_t k, int& w,
                                            const Watchdog& wd) {
     const int slot = k % kItemRing;
     if (k >= kItemRing && !mbar_wait(smem_u32(&r.empty[slot]), (k / kItemRing - 1) & 1, wd))
         return false;
-    w = atomicAdd(counter, 1);
+    const unsigned span = static_cast<unsigned>(c.n_items) + gridDim.x;
+    int old = *reinterpret_cast<volatile int*>(c.ptr);
+    w = c.n_items;
+    // Lock-free: a failed swap means another CTA advanced the counter. The
+    // bound only guards against the impossible; it ends the CTA's work.
+#pragma unroll 1
+    for (int tries = 0; tries < (1 << 20); ++tries) {
+        if (static_cast<unsigned>(old - c.base) > span) {
+            atomicOr(wd.err, kErrSlotReuse);
+            break;
+        }
+        const int prev = atomicCAS(c.ptr, old, old + 1);
+        if (prev == old) {
+            w = old - c.base;
+            break;
+        }
+        old = prev;
+    }
     r.id[slot] = w;
     mbar_arrive(smem_u32(&r.full[slot]));  // release: the index is visible first
     return true;
@@ -241,6 +274,34 @@ __device__ __forceinline__ void bulk_load(uint32_t smem_dst, const void* gsrc, u
             smem_dst),
         "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(bar)
         : "memory");
+}
+
+// Element-wise add of a shared-memory tile into global memory through a tensor
+// map (the addition happens at L2), tracked by the issuing thread's bulk group.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, int c0, int c1,
+                                                  uint32_t smem_src) {
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group"
+        " [%0, {%1, %2}], [%3];" ::"l"(reinterpret_cast<uint64_t>(map)),
+        "r"(c0), "r"(c1), "r"(smem_src)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Waits until the issuing thread's bulk groups have finished READING their
+// shared-memory sources (the buffers may then be reused).
+__device__ __forceinline__ void bulk_wait_read_all() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Waits until the issuing thread's bulk groups have completed entirely.
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy reads (UMMA operands, TMA stores) of the same memory.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {

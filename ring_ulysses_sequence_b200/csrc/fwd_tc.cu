@@ -79,7 +79,7 @@ struct TcArgs {
     void* o;
     float* lse;
     unsigned* status;
-    int* work;         // this launch's work-item counter
+    WorkCounter work;  // this launch's work-item counter
     unsigned long long timeout_ns;
     int H, Hkv, S, P, causal, G;
     MaskSpec mk;       // which keys each query sees
@@ -630,7 +630,6 @@ cudaError_t launch_fwd_tc(const AttnShape& sh, const void* q, const void* k, con
     a.o = o;
     a.lse = lse;
     a.status = ctx.status_word;
-    if ((e = next_work_counter(ctx, &a.work)) != cudaSuccess) return e;
     a.timeout_ns = ctx.watchdog_ns;
     a.H = sh.H;
     a.Hkv = sh.Hkv;
@@ -652,6 +651,7 @@ cudaError_t launch_fwd_tc(const AttnShape& sh, const void* q, const void* k, con
     a.kv_len = len;
     a.owner = step ? sh.owner : 0;
     a.merge = step ? sh.merge : 0;
+    if ((e = next_work_counter(ctx, a.n_items, &a.work)) != cudaSuccess) return e;
     const int grid = std::min(a.n_items, ctx.num_sms);
     if (sh.D == 64) {
         if (sh.mode == kStep) return launch<64, kStep>(a, grid, ctx);

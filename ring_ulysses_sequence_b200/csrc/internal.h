@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "common.cuh"
 #include "rm.h"
 
 namespace rm {
@@ -29,15 +30,20 @@ struct AttnShape {
     int mode;
     int rank, owner;
     int merge;             // mode 2: o, lse hold the running pair; fold the step into it
+    // Backward only: 1 = the two-kernel path (every gradient element written
+    // once: bitwise reproducible); 0 = the fused kernel (dQ by reductions).
+    int deterministic;
 };
 
 // Dynamic work distribution: a persistent kernel's CTAs take work items from a
 // counter in device memory. Each launch uses its own counter slot (rotating
-// over kWorkSlots), zeroed on the launch's stream just before it; at most
-// kWorkSlots launches may be in flight at once.
+// over kWorkSlots), set to a generation-tagged base on the launch's stream
+// just before it; at most kWorkSlots launches may be in flight at once. A
+// launch whose slot another launch re-arms while it runs detects it, stops
+// and raises kErrSlotReuse in the status word (WorkCounter in common.cuh).
 constexpr int kWorkSlots = 256;
-// Zeroes a fresh counter slot on ctx.stream and returns its address.
-cudaError_t next_work_counter(const LaunchCtx& ctx, int** counter);
+// Arms a fresh counter slot on ctx.stream for a launch of n_items items.
+cudaError_t next_work_counter(const LaunchCtx& ctx, int n_items, WorkCounter* counter);
 
 // Forward, bf16, tcgen05 tensor cores (fwd_tc.cu). Modes: see AttnShape::mode.
 cudaError_t launch_fwd_tc(const AttnShape& sh, const void* q, const void* k, const void* v,
@@ -48,7 +54,8 @@ cudaError_t launch_fwd_fp32(const AttnShape& sh, const float* q, const float* k,
 // Backward, bf16 (bwd.cu). delta: Delta [B, H, S] fp32, computed here from o
 // and dout; with mode 2 (one ring step of `rank` against `owner`'s block, the
 // q-side arrays holding the rank's L rows and the k-side ones the block's) it
-// is an input, o is not read, and dq, dk, dv are added to.
+// is an input, o is not read, and dq, dk, dv are added to. sh.deterministic
+// picks the kernels (see AttnShape).
 cudaError_t launch_bwd(const AttnShape& sh, const void* q, const void* k, const void* v,
                        const void* o, const float* lse, const void* dout, float* dq, float* dk,
                        float* dv, float* delta, const LaunchCtx& ctx);

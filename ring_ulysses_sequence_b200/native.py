@@ -10,7 +10,8 @@ import os
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "librm.so")
 
-RM_OK, RM_ERR_INVALID_ARG, RM_ERR_UNSUPPORTED, RM_ERR_CUDA, RM_ERR_TIMEOUT = range(5)
+RM_OK, RM_ERR_INVALID_ARG, RM_ERR_UNSUPPORTED, RM_ERR_CUDA, RM_ERR_TIMEOUT, RM_ERR_SLOT_REUSE = \
+    range(6)
 RM_ORDER_CONTIGUOUS, RM_ORDER_ZIGZAG = 0, 1
 RM_DTYPE_BF16, RM_DTYPE_FP32 = 0, 1
 RM_SEQ_TO_HEAD, RM_HEAD_TO_SEQ = 0, 1
@@ -55,6 +56,8 @@ SIGNATURES = {
     "rm_seq_reorder": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "rm_check_device_status": (_i, [_vp]),
     "rm_set_watchdog_ns": (None, [_u64]),
+    "rm_set_bwd_deterministic": (None, [_i]),
+    "rm_get_bwd_deterministic": (_i, []),
     "rm_watchdog_selftest": (_i, [_u64, _vp]),
     "rm_status_string": (ctypes.c_char_p, [_i]),
     "rm_last_cuda_error": (_i, []),
@@ -261,6 +264,14 @@ def rm_check_device_status(stream=None):
 
 def rm_set_watchdog_ns(ns):
     lib().rm_set_watchdog_ns(int(ns))
+
+
+def rm_set_bwd_deterministic(on):
+    lib().rm_set_bwd_deterministic(int(bool(on)))
+
+
+def rm_get_bwd_deterministic():
+    return int(lib().rm_get_bwd_deterministic())
 
 
 def rm_watchdog_selftest(timeout_ns, stream=None):

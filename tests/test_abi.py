@@ -53,6 +53,7 @@ def test_status_strings(lib):
     assert native.rm_status_string(0) == "ok"
     assert "timed out" in native.rm_status_string(4)
     assert native.rm_status_string(99) == "unknown status"
+    assert "work-counter slots" in native.rm_status_string(native.RM_ERR_SLOT_REUSE)
 
 
 def test_workspace_size(lib):

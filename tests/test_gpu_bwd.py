@@ -2,7 +2,9 @@
 
 The GPU gets O and LSE from its own forward (as a training step would); the
 oracle differentiates exact attention. Tolerances as for O: max-abs 2e-2,
-mean-abs 2e-3 on dQ, dK, dV (fp32 outputs of bf16 inputs).
+mean-abs 2e-3 on dQ, dK, dV (fp32 outputs of bf16 inputs). The default
+backward is the fused kernel; the two-kernel (bitwise reproducible) one is
+checked against it and for determinism.
 """
 import numpy as np
 import pytest
@@ -60,7 +62,17 @@ def test_bwd_shapes_full(B, H, Hkv, S, D, P, order, causal):
     assert float(dk.sum(dim=2).abs().max()) < 0.5
 
 
-def test_bwd_deterministic():
+@pytest.fixture
+def deterministic_bwd():
+    """Selects the two-kernel (bitwise reproducible) backward for one test."""
+    from ring_ulysses_sequence_b200 import native
+    before = native.rm_get_bwd_deterministic()
+    native.rm_set_bwd_deterministic(1)
+    yield
+    native.rm_set_bwd_deterministic(before)
+
+
+def test_bwd_deterministic(deterministic_bwd):
     import ring_ulysses_sequence_b200 as rm
     q, k, v, do = (to_rank_major(t, 4, "zigzag").cuda() for t in _inputs(1, 4, 2, 1024, 128, 77))
     o, lse = rm.ring_attn_fwd(q, k, v, 4, True, "zigzag")
@@ -68,6 +80,42 @@ def test_bwd_deterministic():
     b = rm.ring_attn_bwd(q, k, v, o, lse, do, 4, True, "zigzag")
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("B,H,Hkv,S,D,P,order,causal", [
+    (1, 4, 2, 2048, 128, 4, "zigzag", True),
+    (2, 3, 1, 1024, 64, 2, "contiguous", True),
+    (1, 2, 2, 1024, 128, 4, "zigzag", False),
+])
+def test_fused_and_two_kernel_backward_agree(B, H, Hkv, S, D, P, order, causal):
+    """The default (fused, dQ by reductions) backward and the two-kernel one:
+    dK and dV come from the same per-element arithmetic; dQ differs only in
+    the order of fp32 additions. Both stay within the oracle's tolerance."""
+    import ring_ulysses_sequence_b200 as rm
+    from ring_ulysses_sequence_b200 import native
+    qn, kn, vn, don = _inputs(B, H, Hkv, S, D, 500 + S + H)
+    q, k, v, do = (to_rank_major(t, P, order).cuda() for t in (qn, kn, vn, don))
+    o, lse = rm.ring_attn_fwd(q, k, v, P, causal, order)
+    before = native.rm_get_bwd_deterministic()
+    try:
+        native.rm_set_bwd_deterministic(0)
+        fused = rm.ring_attn_bwd(q, k, v, o, lse, do, P, causal, order)
+        native.rm_set_bwd_deterministic(1)
+        two = rm.ring_attn_bwd(q, k, v, o, lse, do, P, causal, order)
+    finally:
+        native.rm_set_bwd_deterministic(before)
+    torch.cuda.synchronize()
+    assert rm.native.rm_check_device_status() == 0
+    for f, t, name in zip(fused, two, ("dQ", "dK", "dV")):
+        assert_close(f.cpu().numpy(), t.cpu().numpy(), 1e-3, 1e-5, name)
+    rdq, rdkv = oracle.attn_bwd(qn.float(), kn.float(), vn.float(), don.float(), causal)
+    gq, gk, gv = (to_natural(t.cpu(), P, order) for t in fused)
+    for b in range(B):
+        for h in range(H):
+            assert_close(gq[b, h].numpy(), rdq[(b, h)], BF16_MAX_ABS, BF16_MEAN_ABS, f"dQ[{b},{h}]")
+        for g in range(Hkv):
+            assert_close(gk[b, g].numpy(), rdkv[(b, g)][0], BF16_MAX_ABS, BF16_MEAN_ABS, f"dK[{b},{g}]")
+            assert_close(gv[b, g].numpy(), rdkv[(b, g)][1], BF16_MAX_ABS, BF16_MEAN_ABS, f"dV[{b},{g}]")
 
 
 def test_bwd_workload_sampled():

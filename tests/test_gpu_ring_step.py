@@ -197,6 +197,25 @@ def _bwd_inputs(B, H, Hkv, S, D, P, order, causal, seed):
 def test_bwd_steps_sum_to_the_backward(B, H, Hkv, S, D, P, order, causal):
     """P ranks x P steps of rm_ring_attn_bwd_step, in the reverse ring's
     schedule: the oracle's gradients and the one-launch backward."""
+    _bwd_steps_sum(B, H, Hkv, S, D, P, order, causal)
+
+
+@pytest.mark.parametrize("B,H,Hkv,S,D,P,order,causal", [
+    (1, 4, 2, 2048, 128, 4, "zigzag", True),
+    (2, 3, 1, 1024, 64, 2, "zigzag", True),
+])
+def test_bwd_steps_with_the_fused_kernel(B, H, Hkv, S, D, P, order, causal):
+    """The same with the fused backward kernel (dQ added by reductions)."""
+    from ring_ulysses_sequence_b200 import native
+    before = native.rm_get_bwd_deterministic()
+    native.rm_set_bwd_deterministic(0)
+    try:
+        _bwd_steps_sum(B, H, Hkv, S, D, P, order, causal)
+    finally:
+        native.rm_set_bwd_deterministic(before)
+
+
+def _bwd_steps_sum(B, H, Hkv, S, D, P, order, causal):
     import ring_ulysses_sequence_b200 as rm
     (q, k, v, do), (qr, kr, vr, dor, o, lse) = _bwd_inputs(B, H, Hkv, S, D, P, order, causal,
                                                           1400 + S + H)

@@ -38,8 +38,20 @@ def test_concurrent_streams_do_their_own_work():
         assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
 
 
-def test_graph_replay_forward_and_backward():
+@pytest.mark.parametrize("deterministic", [1, 0])
+def test_graph_replay_forward_and_backward(deterministic):
     import ring_ulysses_sequence_b200 as rm
+    before = rm.native.rm_get_bwd_deterministic()
+    rm.native.rm_set_bwd_deterministic(deterministic)
+    try:
+        _graph_replay(deterministic)
+    finally:
+        rm.native.rm_set_bwd_deterministic(before)
+
+
+def _graph_replay(deterministic):
+    import ring_ulysses_sequence_b200 as rm
+    from gpu_util import assert_close
     q, k, v = _inputs(2100)
     do = to_rank_major(make_tensor((1, 8, 2048, 128), 2104, torch.bfloat16, 0.5), 4, "zigzag").cuda()
     o_ref, lse_ref = rm.ring_attn_fwd(q, k, v, 4, True, "zigzag")
@@ -66,4 +78,7 @@ def test_graph_replay_forward_and_backward():
         assert rm.native.rm_check_device_status() == 0
         assert torch.equal(lse, lse_ref) and torch.equal(o, o_ref)
         for g, gr, name in zip(grads, g_ref, ("dQ", "dK", "dV")):
-            assert torch.equal(g, gr), name  # the backward is deterministic
+            if deterministic or name != "dQ":
+                assert torch.equal(g, gr), name  # written once per element
+            else:  # the fused kernel's dQ: reductions in a run-dependent order
+                assert_close(g.cpu().numpy(), gr.cpu().numpy(), 1e-3, 1e-5, name)
