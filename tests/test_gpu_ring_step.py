@@ -353,3 +353,28 @@ def test_step_rejects_bad_arguments():
     with pytest.raises(rm.RMError):                      # fp32: no step variant
         qf = q.float()
         rm.ring_attn_fwd_step(qf, qf, qf, 4, 0, 0)
+
+
+def test_usp_driver_with_one_process_uses_the_library():
+    """ulysses.usp_attn_fwd / usp_attn_bwd with one process (U = R = 1) run the
+    library's pack, unpack, fused step and step-backward kernels end to end:
+    the result is the one-launch forward and backward on the same tokens."""
+    import ring_ulysses_sequence_b200 as rm
+    from ring_ulysses_sequence_b200 import ulysses
+    B, H, Hkv, S, D = 1, 8, 2, 1024, 128
+    q, k, v = (x.cuda() for x in _qkv(B, H, Hkv, S, D, 1700))
+    do = make_tensor((B, H, S, D), 1703, torch.bfloat16, 0.5).cuda()
+    seq = lambda x: x.transpose(1, 2).contiguous()            # [B, S, heads, D]
+    o, ctx = ulysses.usp_attn_fwd(seq(q), seq(k), seq(v), None, None, True, "zigzag")
+    dq, dk, dv = ulysses.usp_attn_bwd(seq(do), ctx, None, None, True, "zigzag")
+    o_ref, lse_ref = rm.ring_attn_fwd(q, k, v, 1, True, "zigzag")
+    g_ref = rm.ring_attn_bwd(q, k, v, o_ref, lse_ref, do, 1, True, "zigzag")
+    torch.cuda.synchronize()
+    assert rm.native.rm_check_device_status() == 0
+    assert o.shape == (B, S, H, D) and o.dtype == torch.float32
+    assert_close(o.transpose(1, 2).cpu().numpy(), o_ref.float().cpu().numpy(), BF16_MAX_ABS,
+                 BF16_MEAN_ABS, what="O")
+    assert_close(ctx.lse.cpu().numpy(), lse_ref.cpu().numpy(), LSE_MAX_ABS, what="LSE")
+    for got, want, name in zip((dq, dk, dv), g_ref, ("dQ", "dK", "dV")):
+        assert_close(got.transpose(1, 2).cpu().numpy(), want.cpu().numpy(), BF16_MAX_ABS,
+                     BF16_MEAN_ABS, what=name)
