@@ -39,11 +39,10 @@
  *     captured a launch keeps that launch's counter: replays of one graph must
  *     not overlap each other, and a replay must not overlap the 256th eager
  *     launch after the capture. A launch whose counter is re-armed by another
- *     one while it runs notices it, stops taking work (its outputs are
- *     undefined) and sets the status word, which rm_check_device_status()
- *     reports as RM_ERR_SLOT_REUSE; the other launch is not disturbed.
- *     (Overlapping replays of one graph re-arm with the same value and cannot
- *     be told apart.)
+ *     one while it runs notices it, stops taking work and sets the status word,
+ *     which rm_check_device_status() reports as RM_ERR_SLOT_REUSE; the outputs
+ *     of both launches are then undefined. (Overlapping replays of one graph
+ *     re-arm with the same value and cannot be told apart.)
  */
 #ifndef RM_H
 #define RM_H

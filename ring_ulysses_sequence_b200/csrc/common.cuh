@@ -200,32 +200,25 @@ struct WorkCounter {
     int n_items;
 };
 
-// Claims the k-th item of this CTA (one thread). The compare-and-swap only
-// advances a counter that still belongs to this launch: a launch that finds
-// its slot re-armed raises kErrSlotReuse and takes no item from the other
-// launch (it publishes n_items, "no more work", and stops).
+// Claims the k-th item of this CTA (one thread). A launch that finds its slot
+// re-armed by another raises kErrSlotReuse and stops (it publishes n_items,
+// "no more work"). Its one claim per CTA has then advanced the other launch's
+// counter, whose results are undefined too; the status word reports it. (A
+// compare-and-swap claim would leave the other launch untouched, but 148
+// producers starting at once serialise on it: it cost several percent on
+// short launches.)
 __device__ __forceinline__ bool item_claim(ItemRing& r, const WorkCounter& c, uint32_t k, int& w,
                                            const Watchdog& wd) {
     const int slot = k % kItemRing;
     if (k >= kItemRing && !mbar_wait(smem_u32(&r.empty[slot]), (k / kItemRing - 1) & 1, wd))
         return false;
+    const int v = atomicAdd(c.ptr, 1) - c.base;
     const unsigned span = static_cast<unsigned>(c.n_items) + gridDim.x;
-    int old = *reinterpret_cast<volatile int*>(c.ptr);
-    w = c.n_items;
-    // Lock-free: a failed swap means another CTA advanced the counter. The
-    // bound only guards against the impossible; it ends the CTA's work.
-#pragma unroll 1
-    for (int tries = 0; tries < (1 << 20); ++tries) {
-        if (static_cast<unsigned>(old - c.base) > span) {
-            atomicOr(wd.err, kErrSlotReuse);
-            break;
-        }
-        const int prev = atomicCAS(c.ptr, old, old + 1);
-        if (prev == old) {
-            w = old - c.base;
-            break;
-        }
-        old = prev;
+    if (static_cast<unsigned>(v) > span) {
+        atomicOr(wd.err, kErrSlotReuse);
+        w = c.n_items;
+    } else {
+        w = v;
     }
     r.id[slot] = w;
     mbar_arrive(smem_u32(&r.full[slot]));  // release: the index is visible first
