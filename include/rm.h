@@ -67,7 +67,8 @@ typedef enum rm_status {
     RM_ERR_UNSUPPORTED = 2,  /* valid request outside the shapes/dtypes built */
     RM_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
     RM_ERR_TIMEOUT = 4,      /* a bounded in-kernel wait ran out */
-    RM_ERR_SLOT_REUSE = 5    /* more launches in flight than work-counter slots */
+    RM_ERR_SLOT_REUSE = 5,   /* more launches in flight than work-counter slots */
+    RM_ERR_SMEM_LAYOUT = 6   /* a kernel's shared-memory layout did not fit its block */
 } rm_status;
 
 /* Token order of the ring ("context parallelism", Last Dictionary: causal
@@ -506,9 +507,12 @@ RM_API rm_status rm_seq_reorder(const void* src, void* dst, int B, int H, int S,
 
 /* Synchronises `stream`, then reads and clears the device status word of the
  * current device. Returns RM_ERR_SLOT_REUSE if a launch found its work counter
- * re-armed by another launch since the last check, else RM_ERR_TIMEOUT if a
- * bounded wait ran out, RM_ERR_CUDA if the synchronisation failed, else
- * RM_OK. */
+ * re-armed by another launch since the last check, else RM_ERR_SMEM_LAYOUT if
+ * a launch found its dynamic shared memory placed too far from a 1024-byte
+ * boundary for its layout (it then returned at once, having written nothing;
+ * only the fused backward checks this, and it has not been seen on sm_100a),
+ * else RM_ERR_TIMEOUT if a bounded wait ran out, RM_ERR_CUDA if the
+ * synchronisation failed, else RM_OK. */
 RM_API rm_status rm_check_device_status(cudaStream_t stream);
 
 /* Limit for every in-kernel wait, in nanoseconds (default 2e9). Applies to

@@ -181,6 +181,7 @@ const char* rm_status_string(rm_status s) {
         case RM_ERR_CUDA: return "CUDA error";
         case RM_ERR_TIMEOUT: return "in-kernel wait timed out";
         case RM_ERR_SLOT_REUSE: return "more launches in flight than work-counter slots";
+        case RM_ERR_SMEM_LAYOUT: return "shared-memory layout did not fit the block";
     }
     return "unknown status";
 }
@@ -206,7 +207,8 @@ rm_status rm_check_device_status(cudaStream_t stream) {
         const unsigned zero = 0;
         e = cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero));
         if (e != cudaSuccess) return cuda_fail(e);
-        return (word & kErrSlotReuse) ? RM_ERR_SLOT_REUSE : RM_ERR_TIMEOUT;
+        if (word & kErrSlotReuse) return RM_ERR_SLOT_REUSE;
+        return (word & kErrSmemLayout) ? RM_ERR_SMEM_LAYOUT : RM_ERR_TIMEOUT;
     }
     return RM_OK;
 }

@@ -98,6 +98,7 @@ struct BwdArgs {
     int rank, owner;
     int q_len;       // rows per head of q, dout, lse, delta, dq: S, or L for one step
     int kv_len;      // rows per head of k, v, dk, dv: S, or L for one step
+    int head_major;  // item order: one head after another (see decode_kv_item)
 };
 
 constexpr int kItemReaders = 9;  // the MMA thread and one lane of each compute warp
@@ -135,11 +136,15 @@ struct KvItem {
 // Key tiles in natural position order, earliest first (causal: they are seen
 // by the most query tiles).
 // One step: the tiles of the owner's block, in slot order; kslot is then the
-// row within the block.
+// row within the block. head_major (whole-ring launches with plain causal or
+// full masks): one head's key tiles after another, so the CTAs running at one
+// time sweep one head's Q and dO, which stay in L2; otherwise (windows, packed
+// documents, one step) the heads of one position are adjacent.
 __device__ __forceinline__ KvItem decode_kv_item(const BwdArgs& a, int w) {
     KvItem it;
-    const int nhu = a.B * a.Hkv;
-    const int unit = w / nhu, hu = w - unit * nhu;
+    const int nhu = a.B * a.Hkv, nu = a.kv_len / kT;
+    const int hu = a.head_major ? w / nu : w % nhu;
+    const int unit = a.head_major ? w - hu * nu : w / nhu;
     it.b = hu / a.Hkv;
     it.g = hu - it.b * a.Hkv;
     if (a.step) {
@@ -582,9 +587,15 @@ struct FCfg {
     static constexpr int kStgOff = kStOff + kStages * kStage;
     static constexpr int kDsOff = kStgOff + kT * 64 * 4;  // own dS^T buffer (D = 64)
     static constexpr int kBarOff = kDsOff + (kDsInStage ? 0 : kT * kT * 2);
-    static constexpr int kSmem = kBarOff + 256 + 1024;
+    static constexpr int kLdOff = kBarOff + 256;   // LSE and Delta of stage s: 2 x 128 fp32
+    static constexpr int kLdStage = 2 * kT * 4;
+    static constexpr int kNeed = kLdOff + kStages * kLdStage;
+    // The layout is 1024-byte aligned; what is allocated beyond kNeed (at most
+    // the 227 KB a block may have) absorbs the dynamic base's misalignment.
+    static constexpr int kSmem = kNeed + 1024 <= 232448 ? kNeed + 1024 : 232448;
+    static constexpr int kSlack = kSmem - kNeed;
 };
-static_assert(FCfg<128>::kSmem <= 232448, "shared memory of the fused backward");
+static_assert(FCfg<128>::kSlack >= 256, "shared memory of the fused backward");
 static_assert(FCfg<64>::kSmem <= 232448, "shared memory of the fused backward");
 
 struct FBars {
@@ -638,10 +649,18 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) ring_bwd_fused_kernel(const __grid_constant__ BwdArgs a) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~static_cast<uintptr_t>(1023));
+    // D = 128 fills the block's shared memory but for 768 bytes: a dynamic base
+    // further than that from a 1024-byte boundary (not seen on sm_100a) makes
+    // the launch return at once with an error in the status word.
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    if (pad > static_cast<uint32_t>(FCfg<D>::kSlack)) {
+        if (threadIdx.x == 0) atomicOr(a.status, kErrSmemLayout);
+        return;
+    }
+    uint8_t* smem = smem_raw + pad;
     FBars& bars = *reinterpret_cast<FBars*>(smem + FCfg<D>::kBarOff);
     const uint32_t k_smem = smem_u32(smem);
+    const uint32_t ld_smem = k_smem + FCfg<D>::kLdOff;  // stage s: LSE[128], Delta[128]
     const uint32_t v_smem = k_smem + FCfg<D>::kTile;
     const uint32_t st_smem = k_smem + FCfg<D>::kStOff;   // stage s: Q, dO
     const uint32_t stg_smem = k_smem + FCfg<D>::kStgOff;  // dQ staging (two 32-column fp32 boxes)
@@ -719,11 +738,13 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_fused_kernel(const __gri
                     const uint32_t base = st_smem + st * FCfg<D>::kStage;
                     const int qrow = (it.b * a.H + h) * a.q_len + qslot;
                     const uint32_t bar = smem_u32(&bars.st_full[st]);
-                    mbar_arrive_expect_tx(bar, FCfg<D>::kStage);
+                    mbar_arrive_expect_tx(bar, FCfg<D>::kStage + FCfg<D>::kLdStage);
                     for (int bx = 0; bx < BCfg<D>::kBoxes; ++bx) {
                         tma_load_2d(base + bx * BCfg<D>::kBox, &a.tm_q, bx * 64, qrow, bar);
                         tma_load_2d(base + FCfg<D>::kTile + bx * BCfg<D>::kBox, &a.tm_do, bx * 64, qrow, bar);
                     }
+                    bulk_load(ld_smem + st * FCfg<D>::kLdStage, a.lse + qrow, kT * 4, bar);
+                    bulk_load(ld_smem + st * FCfg<D>::kLdStage + kT * 4, a.delta + qrow, kT * 4, bar);
                     ++fills;
                 }
             }
@@ -903,8 +924,11 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_fused_kernel(const __gri
                     wq = static_cast<unsigned>(cb.y - cb.x);
                 }
                 const int qrow0 = (it.b * a.H + h) * a.q_len + qslot;
-                const float4* lse4 = reinterpret_cast<const float4*>(a.lse + qrow0 + 64 * wg);
-                const float4* del4 = reinterpret_cast<const float4*>(a.delta + qrow0 + 64 * wg);
+                // LSE and Delta of the tile's queries, loaded with the stage (an
+                // L2 round trip per tile here measured 121 against 108 ms)
+                const float4* lse4 = reinterpret_cast<const float4*>(
+                    smem + FCfg<D>::kLdOff + st * FCfg<D>::kLdStage) + 16 * wg;
+                const float4* del4 = lse4 + kT / 4;
                 ok = mbar_wait(smem_u32(&bars.s_full), s_cnt & 1, wd);
                 if (!ok) break;
                 tc_fence_after();
@@ -919,7 +943,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_fused_kernel(const __gri
                     uint32_t pk[16];
 #pragma unroll
                     for (int c4 = 0; c4 < 8; ++c4) {
-                        const float4 L = __ldg(lse4 + 8 * qq + c4);
+                        const float4 L = lse4[8 * qq + c4];
 #pragma unroll
                         for (int hh = 0; hh < 2; ++hh) {
                             const int c = 4 * c4 + 2 * hh;
@@ -963,7 +987,7 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_fused_kernel(const __gri
                     uint32_t dsk[16];
 #pragma unroll
                     for (int c4 = 0; c4 < 8; ++c4) {
-                        const float4 Dl = __ldg(del4 + 8 * qq + c4);
+                        const float4 Dl = del4[8 * qq + c4];
 #pragma unroll
                         for (int hh = 0; hh < 2; ++hh) {
                             const int c = 4 * c4 + 2 * hh;
@@ -1020,11 +1044,14 @@ struct QItem {
 
 // Query tiles, latest natural position first when causal (the most key tiles).
 // One step: the rank's tiles, latest slot first; slot is then the row within
-// the rank's arrays.
+// the rank's arrays. head_major: one head's query tiles after another (its K
+// and V stay in L2); otherwise the heads of one position are adjacent (the
+// same choice as for the key tiles).
 __device__ __forceinline__ QItem decode_q_item(const BwdArgs& a, int w) {
     QItem it;
-    const int nhu = a.B * a.H;
-    const int unit = w / nhu, hu = w - unit * nhu;
+    const int nhu = a.B * a.H, nq = a.q_len / kT;
+    const int hu = a.head_major ? w / nq : w % nhu;
+    const int unit = a.head_major ? w - hu * nq : w / nhu;
     it.b = hu / a.H;
     it.h = hu - it.b * a.H;
     it.g = it.h / a.G;
@@ -1491,6 +1518,7 @@ cudaError_t launch_bwd(const AttnShape& sh, const void* q, const void* k, const 
     a.owner = step ? sh.owner : 0;
     a.q_len = len;
     a.kv_len = len;
+    a.head_major = (!step && !sh.bounds && !a.mk.window) ? 1 : 0;
     if (!sh.deterministic) {
         if ((e = make_tmap_f32_rows(&a.tm_dq, dq, qrows, sh.D, kT, 32)) != cudaSuccess) return e;
         return sh.D == 64 ? launch_bwd_fused<64>(sh, a, o, dout, delta, dq, ctx)

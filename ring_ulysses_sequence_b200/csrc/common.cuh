@@ -93,7 +93,7 @@ __host__ __device__ __forceinline__ int ceil_div128(int x) { return -((-x) >> 7)
 // Watchdog: every spin-wait is bounded in time.
 // ---------------------------------------------------------------------------
 
-enum : unsigned { kErrTimeout = 1u, kErrSlotReuse = 2u };
+enum : unsigned { kErrTimeout = 1u, kErrSlotReuse = 2u, kErrSmemLayout = 4u };
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;

@@ -84,6 +84,7 @@ struct TcArgs {
     int H, Hkv, S, P, causal, G;
     MaskSpec mk;       // which keys each query sees
     int head_pair;     // 1: tiles are heads (h, h+1) at one slot; 0: one head, slots s, s+128
+    int head_major;    // item order: grouped by KV head (see decode_item)
     int n_units;       // query units per head unit
     int n_head_units;  // B * (head_pair ? H / 2 : H)
     int n_items;
@@ -100,15 +101,31 @@ struct Item {
     int b, h0, h1, g, slot0, slot1, pos0, pos1, rank;
 };
 
-// Work item w -> two query tiles. Items are ordered by the natural position of
-// their queries, latest first when causal (the most key tiles first), with the
-// heads of one position adjacent so that concurrent CTAs share K/V in L2.
+// Work item w -> two query tiles, ordered by the natural position of their
+// queries, latest first when causal (the most key tiles first).
+//   head_major: items grouped by KV head (the head units that read one KV
+//     head), positions inside a group, the group's head units innermost; the
+//     CTAs running at one time then sweep the K/V of one KV head, which stays
+//     in L2 (plain causal or full masks, where a query tile sweeps up to all S
+//     keys and the K/V of every head would not fit).
+//   otherwise: positions outermost, every head of a position adjacent (windows
+//     and packed documents, where a position's keys are few, and one step).
 // One step covers only the launching rank's slots, in slot order.
 template <int kMode>
 __device__ __forceinline__ Item decode_item(const TcArgs& a, int w) {
     Item it;
-    const int unit_rank = w / a.n_head_units;
-    const int hu = w - unit_rank * a.n_head_units;
+    int unit_rank, hu;
+    if (a.head_major) {
+        const int gu = a.head_pair ? a.G / 2 : a.G;  // head units per KV head
+        const int per_group = a.n_units * gu;
+        const int grp = w / per_group;
+        const int rem = w - grp * per_group;
+        unit_rank = rem / gu;
+        hu = grp * gu + (rem - unit_rank * gu);
+    } else {
+        unit_rank = w / a.n_head_units;
+        hu = w - unit_rank * a.n_head_units;
+    }
     const int heads_per_b = a.head_pair ? a.H / 2 : a.H;
     it.b = hu / heads_per_b;
     const int hh = hu - it.b * heads_per_b;
@@ -639,6 +656,7 @@ cudaError_t launch_fwd_tc(const AttnShape& sh, const void* q, const void* k, con
     a.G = sh.H / sh.Hkv;
     a.mk = MaskSpec{static_cast<const int4*>(sh.bounds), sh.S, sh.causal, sh.causal ? sh.window : 0};
     a.head_pair = (a.G % 2 == 0) ? 1 : 0;
+    a.head_major = (!step && !sh.bounds && !a.mk.window) ? 1 : 0;
     a.n_units = a.head_pair ? len / kBM : len / (2 * kBM);
     a.n_head_units = sh.B * (a.head_pair ? sh.H / 2 : sh.H);
     a.n_items = a.n_units * a.n_head_units;

@@ -10,8 +10,8 @@ import os
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "librm.so")
 
-RM_OK, RM_ERR_INVALID_ARG, RM_ERR_UNSUPPORTED, RM_ERR_CUDA, RM_ERR_TIMEOUT, RM_ERR_SLOT_REUSE = \
-    range(6)
+(RM_OK, RM_ERR_INVALID_ARG, RM_ERR_UNSUPPORTED, RM_ERR_CUDA, RM_ERR_TIMEOUT, RM_ERR_SLOT_REUSE,
+ RM_ERR_SMEM_LAYOUT) = range(7)
 RM_ORDER_CONTIGUOUS, RM_ORDER_ZIGZAG = 0, 1
 RM_DTYPE_BF16, RM_DTYPE_FP32 = 0, 1
 RM_SEQ_TO_HEAD, RM_HEAD_TO_SEQ = 0, 1

@@ -54,6 +54,7 @@ def test_status_strings(lib):
     assert "timed out" in native.rm_status_string(4)
     assert native.rm_status_string(99) == "unknown status"
     assert "work-counter slots" in native.rm_status_string(native.RM_ERR_SLOT_REUSE)
+    assert "shared-memory layout" in native.rm_status_string(native.RM_ERR_SMEM_LAYOUT)
 
 
 def test_workspace_size(lib):

@@ -3,8 +3,8 @@
 The GPU gets O and LSE from its own forward (as a training step would); the
 oracle differentiates exact attention. Tolerances as for O: max-abs 2e-2,
 mean-abs 2e-3 on dQ, dK, dV (fp32 outputs of bf16 inputs). The default
-backward is the fused kernel; the two-kernel (bitwise reproducible) one is
-checked against it and for determinism.
+backward is the two-kernel (bitwise reproducible) one, also checked for
+determinism; the fused kernel (dQ by reductions) is checked against it.
 """
 import numpy as np
 import pytest
@@ -88,7 +88,7 @@ def test_bwd_deterministic(deterministic_bwd):
     (1, 2, 2, 1024, 128, 4, "zigzag", False),
 ])
 def test_fused_and_two_kernel_backward_agree(B, H, Hkv, S, D, P, order, causal):
-    """The default (fused, dQ by reductions) backward and the two-kernel one:
+    """The fused backward (dQ by reductions) and the default two-kernel one:
     dK and dV come from the same per-element arithmetic; dQ differs only in
     the order of fp32 additions. Both stay within the oracle's tolerance."""
     import ring_ulysses_sequence_b200 as rm
