@@ -836,9 +836,13 @@ def build_line(out, w, args, world, peaks, peak_src):
                 "kernels": "two kernels, every element written once (rm_set_bwd_deterministic(1), "
                            "the default)",
                 "ms_fused": b.get("ms_fused"), "TFLOPS_fused": b.get("tflops_fused"),
+                "kernels_fused": "one kernel, dQ added by TMA reductions in a run-dependent "
+                                 "order (rm_set_bwd_deterministic(0))",
                 "roofline": {"bound": "tensor", "achieved": b["tflops"],
                              "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                              "frac": b["tflops"] / peaks["bf16_tflops_sustained"],
+                             "frac_fused": (b["tflops_fused"] / peaks["bf16_tflops_sustained"]
+                                            if b.get("tflops_fused") else None),
                              "peak_source": f"{peak_src} bf16_tflops_sustained"}}
     if extra:
         line["extra"] = extra
