@@ -73,6 +73,8 @@ def test_line_carries_the_contract(world):
         rf = extra[name]["roofline"]
         assert rf["frac"] == pytest.approx(rf["achieved"] / rf["peak"]), name
     assert extra["ring_attn_bwd"]["roofline"]["peak"] == 1414.8   # a long step: sustained
+    bwd = extra["ring_attn_bwd"]
+    assert bwd["roofline"]["frac_fused"] == pytest.approx(bwd["TFLOPS_fused"] / 1414.8)
 
 
 def test_line_without_the_forward_keeps_the_extras():
