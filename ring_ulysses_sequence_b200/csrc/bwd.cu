@@ -573,9 +573,9 @@ __global__ void __launch_bounds__(kThreads, 1) ring_bwd_dkdv_kernel(const __grid
 // Q + dO; the dQ staging tile (128 rows x 64 fp32, two 32-column boxes with
 // the 128-byte swizzle). dS^T (128 x 128 bf16, laid out like a TMA tile) goes
 // over the stage's dO once dV has read it when D = 128 (dO is then exactly
-// its size); with D = 64 it has a buffer of its own. LSE and Delta come
-// straight from global memory (every thread of a warpgroup reads the same 64
-// values).
+// its size); with D = 64 it has a buffer of its own. The LSE and Delta of
+// each stage's 128 queries are loaded with it into the last 2 KB (every
+// thread of a warpgroup reads the same 64 values of each).
 constexpr int kDsBox = kT * 128;  // one 64-column box of the dS^T tile; one 32-column fp32 box
 
 template <int D>
