@@ -724,7 +724,7 @@ def build_line(out, w, args, world, peaks, peak_src):
             "pct_of_peak_basis": f"{peak_src} bf16 GEMM ceiling {peak} TFLOPS "
                                  "(torch.matmul 8192^3 burst on this pool's B200s)",
             "pct_of_datasheet_dense_peak": 100.0 * achieved / 2250.0,
-            "roofline": {"bound": "tensor", "kernel": "ring_fwd_tc_kernel<128, false>",
+            "roofline": {"bound": "tensor", "kernel": "ring_fwd_tc_kernel<128, 0>",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak,
                          "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)",
