@@ -25,3 +25,14 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(params=[1, 0], ids=["two_kernels", "fused"])
+def bwd_kernels(request):
+    """Runs a backward test with each backward path: 1 the two kernels (the
+    default), 0 the fused kernel (dQ by reductions); the switch is restored."""
+    from ring_ulysses_sequence_b200 import native
+    before = native.rm_get_bwd_deterministic()
+    native.rm_set_bwd_deterministic(request.param)
+    yield request.param
+    native.rm_set_bwd_deterministic(before)

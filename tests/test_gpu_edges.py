@@ -35,7 +35,7 @@ def _padded_len(S_real, P, order):
     (1, 2, "zigzag", True),
     (1500, 2, "contiguous", False),
 ])
-def test_ragged_length_padded_and_masked(S_real, P, order, causal):
+def test_ragged_length_padded_and_masked(S_real, P, order, causal, bwd_kernels):
     import ring_ulysses_sequence_b200 as rm
     B, H, Hkv, D = 1, 4, 2, 128
     S = _padded_len(S_real, P, order)

@@ -107,7 +107,7 @@ def test_varlen_result_independent_of_P_and_order():
     ([0, 128, 256, 640, 1024], False, 0),
     ([0, 1, 1, 2, 300, 1023, 1024], True, 150),
 ])
-def test_varlen_backward(cu, causal, window):
+def test_varlen_backward(cu, causal, window, bwd_kernels):
     import ring_ulysses_sequence_b200 as rm
     B, H, Hkv, S, D, P, order = 1, 4, 2, 1024, 128, 4, "zigzag"
     qn, kn, vn = _qkv(B, H, Hkv, S, D, 1600 + len(cu), torch.bfloat16)
@@ -145,7 +145,7 @@ def test_varlen_batched_and_d64(B, H, Hkv, D, causal):
     _check(q, k, v, 4, "zigzag", cu, causal)
 
 
-def test_varlen_backward_d64_batched():
+def test_varlen_backward_d64_batched(bwd_kernels):
     import ring_ulysses_sequence_b200 as rm
     B, H, Hkv, S, D, P, order, cu = 2, 2, 1, 512, 64, 2, "contiguous", [0, 100, 356, 512]
     qn, kn, vn = _qkv(B, H, Hkv, S, D, 1800, torch.bfloat16)

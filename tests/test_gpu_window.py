@@ -113,7 +113,7 @@ def gpu_grads(qn, kn, vn, don, P, order, W):
     (2, 3, 1, 512, 64, 2, "zigzag", 128),
     (1, 2, 1, 2048, 128, 8, "zigzag", 700),
 ])
-def test_window_backward(B, H, Hkv, S, D, P, order, W):
+def test_window_backward(B, H, Hkv, S, D, P, order, W, bwd_kernels):
     q, k, v = _qkv(B, H, Hkv, S, D, 900 + W, torch.bfloat16)
     do = make_tensor((B, H, S, D), 950 + W, torch.bfloat16, 0.5)
     dq, dk, dv = gpu_grads(q, k, v, do, P, order, W)
@@ -143,7 +143,7 @@ def test_window_workload_sampled_rows():
 
 
 @pytest.mark.parametrize("W", [1, 100, 257])
-def test_window_d64_forward_and_backward(W):
+def test_window_d64_forward_and_backward(W, bwd_kernels):
     B, H, Hkv, S, D, P, order = 1, 4, 2, 1024, 64, 4, "zigzag"
     q, k, v = _qkv(B, H, Hkv, S, D, 1900 + W, torch.bfloat16)
     _check_fwd(q, k, v, P, order, W)
