@@ -99,7 +99,7 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
 
-    def __init__(self, device_index, period_s=0.05):
+    def __init__(self, device_index, period_s=0.01):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period = period_s
         self._stop = threading.Event()
